@@ -1,0 +1,337 @@
+// CPU oracle for the FP8 (E4M3) attention forward with P-cast scale S and KV order.
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link,
+// load or call this file: only tests/, __graft_entry__.smoke() and bench.py's
+// CPU-baseline / reference leg use it.  It shares no code with the CUDA path.
+//
+// Source of truth: "P-Cast Precision in FP8 Attention: Sink-Induced Collapse and
+// the Optimality of S=2^8" (arXiv 2606.06521), as summarised on gist.science
+// (pt / de / hi pages).  Section names below are those pages' sections.
+//
+// Plain, slow, obviously sequential code:
+//   * e4m3_*     : the E4M3 number format (Problem statement: 3-bit mantissa;
+//                  Methodology: round-to-zero threshold 2^-10; Optimality of
+//                  S=256, condition 3: normal floor 2^-6, largest finite 448).
+//   * attn_exact : float64 softmax attention on the decoded E4M3 inputs.
+//   * attn_emulate : the FP8 pipeline, KV block by KV block, in the order the
+//                  online softmax visits the blocks (Problem statement:
+//                  running max m, KV iteration order, static scale S applied
+//                  before the cast and divided back out in the epilogue).
+//   * collapse_logits : the same online softmax on given scaled logits, used
+//                  for the closed-form underflow fraction F(Delta,S)
+//                  (Methodology, theoretical framework).
+// All FP32 sums run left to right in the order stated at each loop.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+#include <omp.h>
+
+namespace {
+
+const float kNegInf = -std::numeric_limits<float>::infinity();
+
+// ---------------------------------------------------------------- E4M3 ------
+// OCP FP8 E4M3 ("fn" variant): sign, 4-bit exponent (bias 7), 3-bit mantissa.
+// No infinities; S.1111.111 is NaN.  e = 0 is subnormal: m * 2^-9.
+double e4m3_value(uint8_t c) {
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+    double mag = (e == 0) ? std::ldexp((double)m, -9) : std::ldexp((double)(8 + m), e - 10);
+    return s ? -mag : mag;
+}
+
+// Round-to-nearest-even onto the E4M3 grid, saturating finite values above the
+// largest finite 448 (and infinities) to +-448; NaN -> 0x7F.
+uint8_t e4m3_encode(float x) {
+    if (std::isnan(x)) return 0x7F;
+    uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+    double a = std::fabs((double)x);
+    if (a > 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    // grid spacing at a: subnormal range (a < 2^-6) has spacing 2^-9; in the
+    // binade [2^e, 2^(e+1)) with e >= -6 the spacing is 2^(e-3).
+    int ex;
+    std::frexp(a, &ex);             // a = f * 2^ex, f in [0.5, 1)  ->  floor(log2 a) = ex-1
+    int e = ex - 1;
+    double spacing = (e < -6) ? std::ldexp(1.0, -9) : std::ldexp(1.0, e - 3);
+    double r = std::nearbyint(a / spacing);   // default rounding mode: ties to even
+    double val = r * spacing;
+    if (val == 0.0) return sign;
+    if (val > 448.0) return sign | 0x7E;      // cannot happen after the a > 448 test
+    int vex;
+    std::frexp(val, &vex);
+    int ve = vex - 1;
+    uint8_t code;
+    if (ve < -6) {
+        code = (uint8_t)(val / std::ldexp(1.0, -9));            // subnormal: m = val / 2^-9
+    } else {
+        int m = (int)(val / std::ldexp(1.0, ve) * 8.0) - 8;      // val = 2^ve (1 + m/8)
+        code = (uint8_t)(((ve + 7) << 3) | m);
+    }
+    return sign | code;
+}
+
+float g_dec[256];
+struct DecInit {
+    DecInit() { for (int c = 0; c < 256; ++c) g_dec[c] = (float)e4m3_value((uint8_t)c); }
+} g_dec_init;
+
+// BF16 round-to-nearest-even of a finite float, returned as a float.
+float bf16_rne(float x) {
+    uint32_t u;
+    std::memcpy(&u, &x, 4);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    u &= 0xFFFF0000u;
+    float y;
+    std::memcpy(&y, &u, 4);
+    return y;
+}
+
+struct Shape {
+    int B, H, Hkv, N, d;
+};
+
+// (b, h, i) of a global query row index r in [0, B*H*N)
+inline void row_coords(const Shape& s, int64_t r, int& b, int& h, int& i) {
+    i = (int)(r % s.N);
+    int64_t bh = r / s.N;
+    h = (int)(bh % s.H);
+    b = (int)(bh / s.H);
+}
+
+// Online softmax state of one query row (Problem statement: running max m; the
+// row sum l is accumulated from the FP32 probabilities before the cast).
+struct RowState {
+    float m = kNegInf;
+    float l = 0.0f;
+};
+
+// One KV block of the FP8 pipeline for one row.
+//   s[j]  : scaled logits (FP32), -inf where masked
+//   on return: pt[j] = E4M3 code of fl32(S * p_j); alpha = rescale of the old state
+//   collapse counted for j_global >= n_sink with p_j > 0 and code magnitude 0.
+// Returns the number of collapsed entries.
+int softmax_block(const float* s, int n, int j0, int n_sink, float S, RowState& st,
+                  uint8_t* pt, float* alpha_out) {
+    float mblk = kNegInf;
+    for (int j = 0; j < n; ++j) mblk = std::fmax(mblk, s[j]);
+    float m_new = std::fmax(st.m, mblk);
+    float alpha;
+    if (m_new == kNegInf) alpha = 1.0f;          // nothing visible yet
+    else if (st.m == kNegInf) alpha = 0.0f;      // first visible block
+    else alpha = std::exp(st.m - m_new);
+    float rowsum = 0.0f;
+    int collapsed = 0;
+    for (int j = 0; j < n; ++j) {
+        float p = (s[j] == kNegInf) ? 0.0f : std::exp(s[j] - m_new);
+        rowsum += p;
+        float t = S * p;                          // fl32(S * p)
+        uint8_t c = e4m3_encode(t);
+        pt[j] = c;
+        if (p > 0.0f && (c & 0x7F) == 0 && (j0 + j) >= n_sink) ++collapsed;
+    }
+    st.l = alpha * st.l + rowsum;
+    st.m = m_new;
+    *alpha_out = alpha;
+    return collapsed;
+}
+
+inline bool block_has_sink(int blk, int block_n, int n_sink) { return blk * block_n < n_sink; }
+
+}  // namespace
+
+extern "C" {
+
+// ---- codec entry points -----------------------------------------------------
+double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
+uint8_t oracle_e4m3_encode(float x) { return e4m3_encode(x); }
+float oracle_bf16_rne(float x) { return bf16_rne(x); }
+
+// out[i] = E4M3(fl32(S * x[i]))
+void oracle_e4m3_scale_cast(const float* x, uint8_t* out, int64_t n, float S) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_encode(S * x[i]);
+}
+
+// out[i] = E4M3(fl32(S * bitcast<float>(first + i)))  (exhaustive bit-pattern sweeps)
+void oracle_e4m3_scale_cast_bits(uint64_t first, int64_t n, float S, uint8_t* out) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t u = (uint32_t)(first + (uint64_t)i);
+        float x;
+        std::memcpy(&x, &u, 4);
+        out[i] = e4m3_encode(S * x);
+    }
+}
+
+// ---- float64 exact attention on decoded E4M3 inputs ------------------------
+// O*[r, :] = sum_j softmax_j(scale * q_i . k_j) v_j, causal: j <= i;
+// query head h reads kv head h / (H / Hkv).  rows == NULL: all B*H*N rows.
+int oracle_attn_exact(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
+                      int B, int H, int Hkv, int N, int d, int causal, double scale,
+                      const int64_t* rows, int64_t nrows, double* O, int nthreads) {
+    if (H % Hkv) return -1;
+    Shape sh{B, H, Hkv, N, d};
+    if (!rows) nrows = (int64_t)B * H * N;
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+    const int group = H / Hkv;
+    #pragma omp parallel
+    {
+        std::vector<double> s(N), q(d), acc(d);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t t = 0; t < nrows; ++t) {
+            int64_t r = rows ? rows[t] : t;
+            int b, h, i;
+            row_coords(sh, r, b, h, i);
+            const uint8_t* qp = Q + (((int64_t)b * H + h) * N + i) * d;
+            const int64_t kvbase = (((int64_t)b * Hkv + h / group) * N) * d;
+            for (int k = 0; k < d; ++k) q[k] = e4m3_value(qp[k]);
+            int jend = causal ? i + 1 : N;
+            double mx = -std::numeric_limits<double>::infinity();
+            for (int j = 0; j < jend; ++j) {
+                const uint8_t* kp = K + kvbase + (int64_t)j * d;
+                double dot = 0.0;
+                for (int k = 0; k < d; ++k) dot += q[k] * e4m3_value(kp[k]);
+                s[j] = scale * dot;
+                if (s[j] > mx) mx = s[j];
+            }
+            double sum = 0.0;
+            for (int k = 0; k < d; ++k) acc[k] = 0.0;
+            for (int j = 0; j < jend; ++j) {
+                double e = std::exp(s[j] - mx);
+                sum += e;
+                const uint8_t* vp = V + kvbase + (int64_t)j * d;
+                for (int k = 0; k < d; ++k) acc[k] += e * e4m3_value(vp[k]);
+            }
+            for (int k = 0; k < d; ++k) O[t * d + k] = acc[k] / sum;
+        }
+    }
+    return 0;
+}
+
+// ---- FP8 pipeline emulation -------------------------------------------------
+// Per query row (FP32 throughout):
+//   m = -inf, l = 0, acc = 0
+//   for each KV block in the visiting order (forward: 0..last, reverse: last..0;
+//   last = floor(i / block_n) when causal, else N/block_n - 1):
+//     s_j    = fl32(scale * fl32(sum_k q_k k_jk))   (k ascending), -inf if j > i (causal)
+//     m'     = max(m, max_j s_j)
+//     alpha  = exp(m - m')    (0 when m = -inf; 1 when m' = -inf)
+//     p_j    = exp(s_j - m')  (0 where s_j = -inf)
+//     l      = alpha * l + (sum_j p_j)               (j ascending)
+//     pt_j   = E4M3_RNE_satfinite(fl32(S * p_j))
+//     collapse if p_j > 0, pt_j == 0 and j >= n_sink
+//     acc_k  = alpha * acc_k + sum_j dec(pt_j) * dec(v_jk)   (j ascending)
+//     m = m'
+//   O_k = acc_k / fl32(S * l), then BF16 RNE when o_bf16.
+// Outputs: O [nrows, d] (float), collapse_rows [nrows] (nullable),
+// collapse_totals[2] = {entries in KV blocks holding a sink key, entries in the
+// other blocks} (nullable, accumulated).
+int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
+                        int B, int H, int Hkv, int N, int d, int causal, float scale, float S,
+                        int kv_order, int block_n, int n_sink, int o_bf16,
+                        const int64_t* rows, int64_t nrows,
+                        float* O, uint32_t* collapse_rows, uint64_t* collapse_totals,
+                        int nthreads) {
+    if (H % Hkv || block_n <= 0 || N % block_n) return -1;
+    Shape sh{B, H, Hkv, N, d};
+    if (!rows) nrows = (int64_t)B * H * N;
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+    const int group = H / Hkv;
+    const int nblocks = N / block_n;
+    uint64_t tot_sink = 0, tot_other = 0;
+    #pragma omp parallel reduction(+ : tot_sink, tot_other)
+    {
+        std::vector<float> q(d), acc(d), s(block_n), vdec((size_t)block_n * d);
+        std::vector<uint8_t> pt(block_n);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t t = 0; t < nrows; ++t) {
+            int64_t r = rows ? rows[t] : t;
+            int b, h, i;
+            row_coords(sh, r, b, h, i);
+            const uint8_t* qp = Q + (((int64_t)b * H + h) * N + i) * d;
+            const int64_t kvbase = (((int64_t)b * Hkv + h / group) * N) * d;
+            for (int k = 0; k < d; ++k) q[k] = g_dec[qp[k]];
+            for (int k = 0; k < d; ++k) acc[k] = 0.0f;
+            RowState st;
+            uint32_t row_collapse = 0;
+            const int last = causal ? i / block_n : nblocks - 1;
+            for (int step = 0; step <= last; ++step) {
+                const int blk = (kv_order == 0) ? step : last - step;
+                const int j0 = blk * block_n;
+                for (int jj = 0; jj < block_n; ++jj) {
+                    int j = j0 + jj;
+                    if (causal && j > i) { s[jj] = kNegInf; continue; }
+                    const uint8_t* kp = K + kvbase + (int64_t)j * d;
+                    float dot = 0.0f;
+                    for (int k = 0; k < d; ++k) dot += q[k] * g_dec[kp[k]];
+                    s[jj] = scale * dot;
+                }
+                float alpha;
+                int c = softmax_block(s.data(), block_n, j0, n_sink, S, st, pt.data(), &alpha);
+                row_collapse += (uint32_t)c;
+                if (block_has_sink(blk, block_n, n_sink)) tot_sink += (uint64_t)c;
+                else tot_other += (uint64_t)c;
+                for (int k = 0; k < d; ++k) acc[k] = alpha * acc[k];
+                for (int jj = 0; jj < block_n; ++jj) {
+                    float pv = g_dec[pt[jj]];
+                    if (pv == 0.0f) continue;   // adds exactly +0 (v is finite)
+                    const uint8_t* vp = V + kvbase + (int64_t)(j0 + jj) * d;
+                    for (int k = 0; k < d; ++k) acc[k] += pv * g_dec[vp[k]];
+                }
+            }
+            float denom = S * st.l;
+            for (int k = 0; k < d; ++k) {
+                float o = acc[k] / denom;
+                O[t * d + k] = o_bf16 ? bf16_rne(o) : o;
+            }
+            if (collapse_rows) collapse_rows[t] = row_collapse;
+        }
+    }
+    if (collapse_totals) {
+        collapse_totals[0] += tot_sink;
+        collapse_totals[1] += tot_other;
+    }
+    return 0;
+}
+
+// ---- online softmax on given scaled logits (closed-form pins) ---------------
+// logits [nrows, N] are the s_j above.  Non-causal.  Returns per-row collapse
+// counts and accumulates collapse_totals[2] as in oracle_attn_emulate.
+int oracle_collapse_logits(const float* logits, int64_t nrows, int N, int block_n, int n_sink,
+                           float S, int kv_order, uint32_t* collapse_rows,
+                           uint64_t* collapse_totals, int nthreads) {
+    if (block_n <= 0 || N % block_n) return -1;
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+    const int nblocks = N / block_n;
+    uint64_t tot_sink = 0, tot_other = 0;
+    #pragma omp parallel reduction(+ : tot_sink, tot_other)
+    {
+        std::vector<uint8_t> pt(block_n);
+        #pragma omp for schedule(static)
+        for (int64_t r = 0; r < nrows; ++r) {
+            RowState st;
+            uint32_t rc = 0;
+            for (int step = 0; step < nblocks; ++step) {
+                int blk = (kv_order == 0) ? step : nblocks - 1 - step;
+                float alpha;
+                int c = softmax_block(logits + r * (int64_t)N + (int64_t)blk * block_n, block_n,
+                                      blk * block_n, n_sink, S, st, pt.data(), &alpha);
+                rc += (uint32_t)c;
+                if (block_has_sink(blk, block_n, n_sink)) tot_sink += (uint64_t)c;
+                else tot_other += (uint64_t)c;
+            }
+            if (collapse_rows) collapse_rows[r] = rc;
+        }
+    }
+    if (collapse_totals) {
+        collapse_totals[0] += tot_sink;
+        collapse_totals[1] += tot_other;
+    }
+    return 0;
+}
+
+}  // extern "C"
