@@ -1,0 +1,136 @@
+/* fp8attn.h - C ABI of the B200 (sm_100a) FP8 attention forward with P-cast
+ * scale S and selectable KV-block order.
+ *
+ * What the operation is (P-Cast Precision in FP8 Attention: Sink-Induced
+ * Collapse and the Optimality of S=2^8, arXiv 2606.06521, gist.science
+ * summary, section 1 "Problem statement"): a FlashAttention-style forward
+ * pass on E4M3 operands whose online softmax keeps a running row max m,
+ * multiplies each probability tile P by a static scale S, casts S*P to E4M3
+ * for the P.V product, and divides S back out in the epilogue.  The order in
+ * which the online softmax visits the KV blocks (forward 0..N or reverse N..0)
+ * is a run-time choice; section 2 "Optimisation 1" shows that the reverse order
+ * keeps the attention sink from inflating m before the other blocks are cast.
+ * "P-collapse" (section 1) is a non-sink P that is nonzero in FP32 but 0 after
+ * the cast; the kernel can count it.
+ *
+ * Per query row i (query head h, kv head h / (H / H_kv)):
+ *   for each KV block of block_n keys, in the chosen order:
+ *     s_j  = scale * q_i . k_j        (FP32 accumulate of E4M3 products)
+ *     m'   = max(m, max_j s_j),  alpha = exp(m - m')
+ *     p_j  = exp(s_j - m')            (FP32)
+ *     l    = alpha * l + sum_j p_j    (row sum from the FP32 P, before the cast)
+ *     pt_j = E4M3_RNE_satfinite(S * p_j)
+ *     acc  = alpha * acc + sum_j pt_j v_j   (E4M3 x E4M3, FP32 accumulate)
+ *     m    = m'
+ *   O_i = acc / (S * l)
+ * Causal: key j is visible to query i iff j <= i (square prefill, no offset).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     never frees or retains them and allocates no device memory.
+ *   - All work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream).  A return of FP8ATTN_OK means "validated and launched".
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns a negative status and touches no device memory.
+ *     fp8attn_last_error() then gives a one-line reason (per host thread).
+ *   - E4M3 means the OCP FP8 E4M3 ("fn") byte encoding, one byte per element.
+ */
+#ifndef FP8ATTN_H
+#define FP8ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* fp8attn_stream_t;
+
+typedef enum {
+  FP8ATTN_OK = 0,
+  FP8ATTN_EINVAL = -1,        /* an argument is out of range or misaligned */
+  FP8ATTN_EUNSUPPORTED = -2,  /* a valid request this build does not serve (d, block_n) */
+  FP8ATTN_ECUDA = -3,         /* a CUDA runtime / driver call failed */
+  FP8ATTN_ETIMEOUT = -4       /* reported through status_word: a bounded wait expired */
+} fp8attn_status;
+
+enum { FP8ATTN_KV_FORWARD = 0, FP8ATTN_KV_REVERSE = 1 };
+enum { FP8ATTN_O_BF16 = 0, FP8ATTN_O_F32 = 1 };
+
+/* fp8_attn_fwd - the attention forward above, square self-attention, H_kv = H,
+ * O in BF16, KV block 128.
+ *
+ *   Q, K, V   E4M3 [B, H, N, d] contiguous (d fastest), 16-byte aligned.
+ *   O         BF16 [B, H, N, d] contiguous, 16-byte aligned (written).
+ *   B, H, N   batch, heads, sequence length; B*H*N == 0 is a no-op.
+ *   d         head dimension, 64 or 128.
+ *   causal    0 or 1.
+ *   scale     softmax scale (finite, > 0), usually 1/sqrt(d).
+ *   S         P-cast scale (finite, > 0).  S > 448 is accepted: S*P then
+ *             saturates at 448 (the overflow the paper warns of for 512).
+ *   kv_order  FP8ATTN_KV_FORWARD or FP8ATTN_KV_REVERSE.
+ *   n_sink    keys j < n_sink are sinks and are never counted (0 <= n_sink <= N).
+ *   collapse_ctr  NULL: no counting (the faster kernel variant).  Otherwise a
+ *             device uint64 that the kernel ADDS the number of collapsed
+ *             entries to (the caller zeroes it).
+ * Returns an fp8attn_status. */
+int fp8_attn_fwd(const void* Q, const void* K, const void* V, void* O,
+                 int B, int H, int N, int d, int causal, float scale, float S,
+                 int kv_order, int n_sink, unsigned long long* collapse_ctr,
+                 fp8attn_stream_t stream);
+
+/* Full parameter set (same operation; see fp8_attn_fwd for shared fields). */
+typedef struct {
+  const void* Q;          /* E4M3 [B, H,    N, d] */
+  const void* K;          /* E4M3 [B, H_kv, N, d] */
+  const void* V;          /* E4M3 [B, H_kv, N, d] */
+  void* O;                /* [B, H, N, d], dtype o_dtype */
+  int B, H, H_kv, N, d;   /* H % H_kv == 0; query head h reads kv head h / (H / H_kv) */
+  int causal;
+  float scale, S;
+  int kv_order, n_sink;
+  int o_dtype;            /* FP8ATTN_O_BF16 (RNE) or FP8ATTN_O_F32 */
+  int block_n;            /* KV block: 0 (= 128), 64 or 128.  N need not be a multiple:
+                             the last block then holds the remaining keys. */
+  unsigned long long* collapse_ctr;      /* nullable; += all collapsed entries */
+  unsigned long long* collapse_sink_ctr; /* nullable; += those in KV blocks holding a
+                                            sink key (requires collapse_ctr) */
+  unsigned int* collapse_rows;           /* nullable; [B, H, N] per-row counts, written
+                                            (requires collapse_ctr) */
+  unsigned int* status_word;             /* nullable device word; a kernel whose bounded
+                                            wait expires writes a nonzero code here and
+                                            leaves O incomplete */
+  unsigned long long timeout_ns;         /* bound of each wait; 0 = 2 s */
+} fp8attn_params;
+
+int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream);
+
+/* fp8_e4m3_scale_cast - out[i] = E4M3_RNE_satfinite(fl32(S * P[i])) for i < n,
+ * with the device conversion routine the attention kernel uses for S*P
+ * (P-cast paper, section 2 "Optimality of S=256": the scaling happens in FP32,
+ * then the round-to-nearest cast).  P: device float[n]; out: device uint8[n];
+ * both 16-byte aligned.  S finite (any sign).  NaN -> 0x7F, |x| > 448 -> +-448. */
+int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
+                        fp8attn_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fp8attn_status_string(int status);
+
+/* Reason for the last non-OK return on this host thread ("" if none). */
+const char* fp8attn_last_error(void);
+
+/* Decoded device status word value ("" for 0). */
+const char* fp8attn_device_status_string(unsigned int word);
+
+/* ABI version of this header (major * 100 + minor). */
+int fp8attn_version(void);
+
+/* sizeof(fp8attn_params) as compiled into the library (binding layout check). */
+size_t fp8attn_params_sizeof(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8ATTN_H */

@@ -1,0 +1,638 @@
+// fp8_attn_fwd.cu - FP8 (E4M3) attention forward for B200 (sm_100a) with the
+// P-cast scale S and a run-time KV-block order, behind the C ABI of
+// include/fp8attn.h.
+//
+// Method: "P-Cast Precision in FP8 Attention: Sink-Induced Collapse and the
+// Optimality of S=2^8" (arXiv 2606.06521, gist.science summary).  Section 1
+// (Problem statement) fixes what is computed: an online softmax with running
+// max m over KV blocks visited forward (0..N) or in reverse (N..0), the
+// probability tile multiplied by a static S and cast to E4M3 for P.V, and S
+// divided back out in the epilogue.  Section 2 (Optimisation 1) is why the
+// order is a parameter; the collapse counter measures the P-collapse of
+// section 1.
+//
+// One CTA owns one 128-row query tile of one (batch, head) and runs four
+// warp-specialised roles (two CTAs share an SM so that one CTA's softmax
+// overlaps the other's tensor-core work):
+//   warp 4     TMA producer: Q tile once, then K and V tiles of each KV block in
+//              visiting order into a 2-stage ring (3-D tensor maps, so a ragged
+//              last block reads zeros past N).
+//   warp 5     MMA issuer: S = Q K^T into TMEM (tcgen05 kind::f8f6f4, M=128,
+//              N=block_n, K=32 per instruction), then O += P~ V into TMEM
+//              (V as an MN-major operand).  Owns the TMEM allocation.
+//   warps 0-3  softmax, one thread per query row: tcgen05.ld of its S row, row
+//              max, exp2, FP32 row sum, S-multiply, E4M3 cast into a swizzled
+//              shared-memory P~ tile, collapse count, the O rescale in TMEM when a
+//              row max changed, and the epilogue O / (S l).
+// Every mbarrier wait is bounded in time: on expiry the CTA sets a shared
+// abort flag, every role leaves its loop, in-flight copies and MMAs are
+// drained, TMEM is freed and the status word (if given) records where.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fp8attn.h"
+#include "sm100.cuh"
+
+namespace fp8attn {
+
+constexpr int BM = 128;         // query rows per CTA (= MMA M, = TMEM lanes)
+constexpr int NSTAGE = 2;       // K/V ring depth
+constexpr int NTHREADS = 192;   // 4 softmax warps + TMA warp + MMA warp
+constexpr float LOG2E = 1.4426950408889634f;
+
+// device status codes (status_word): 0x100 | where the wait gave up
+enum : uint32_t {
+  WAIT_PROD_KV_EMPTY = 1,
+  WAIT_MMA_Q = 2,
+  WAIT_MMA_K = 3,
+  WAIT_MMA_S_FREE = 4,
+  WAIT_MMA_V = 5,
+  WAIT_MMA_P = 6,
+  WAIT_SM_S_FULL = 7,
+  WAIT_SM_O_DONE = 8,
+  WAIT_EPI_O_DONE = 9,
+};
+
+struct KParams {
+  int B, H, Hkv, N, group;
+  int causal, kv_order, n_sink;
+  int num_q_tiles;
+  float scale_log2;   // scale * log2(e)
+  float S;
+  void* O;
+  unsigned long long* ctr;
+  unsigned long long* ctr_sink;
+  unsigned int* rows;
+  unsigned int* status;
+  unsigned long long timeout_ns;
+};
+
+template <int D, int BN>
+struct Smem {
+  static constexpr int Q = 0;
+  static constexpr int K = Q + BM * D;
+  static constexpr int V = K + NSTAGE * BN * D;
+  static constexpr int P = V + NSTAGE * BN * D;
+  static constexpr int BAR = P + BM * BN;
+  // barriers: q_full, k_full[2], v_full[2], kv_empty[2], s_full, s_free, p_full, o_done, drain
+  static constexpr int NBAR = 1 + 3 * NSTAGE + 5;
+  static constexpr int MISC = BAR + 8 * NBAR;   // tmem base slot, abort flag
+  static constexpr int BYTES = MISC + 16;
+  // slack to align the base to 1024, and at least 80 KB so that no more than two
+  // CTAs share an SM: two 256-column TMEM allocations fill the SM's 512 columns
+  static constexpr int ALLOC = (BYTES + 1024 > 80 * 1024) ? BYTES + 1024 : 80 * 1024;
+  static constexpr uint32_t TMEM_COLS = 256;    // S: BN columns, O: D columns
+  static_assert(BN + D <= (int)TMEM_COLS, "TMEM budget");
+};
+
+__device__ __forceinline__ int kv_block_at(int t, int T, int order) {
+  return order == FP8ATTN_KV_FORWARD ? t : T - 1 - t;
+}
+
+template <int D, int BN, bool OUT_BF16, bool COUNT>
+__global__ void __launch_bounds__(NTHREADS, 2)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const KParams p) {
+  using L = Smem<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + L::Q, sK = sbase + L::K, sV = sbase + L::V, sP = sbase + L::P;
+  const uint32_t bar0 = sbase + L::BAR;
+  const uint32_t bar_q_full = bar0;
+  auto bar_k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
+  auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
+  const uint32_t bar_s_full = bar0 + 8u * (1 + 3 * NSTAGE);
+  const uint32_t bar_s_free = bar_s_full + 8;
+  const uint32_t bar_p_full = bar_s_full + 16;
+  const uint32_t bar_o_done = bar_s_full + 24;
+  const uint32_t bar_drain = bar_s_full + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = p.causal ? (p.num_q_tiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % p.H, b = bh / p.H;
+  const int bkv = b * p.Hkv + h / p.group;
+  const int q0 = tile * BM;
+  const int last_row = min(q0 + BM - 1, p.N - 1);
+  const int T = p.causal ? (last_row / BN + 1) : ((p.N + BN - 1) / BN);
+  const WaitCtl ctl{abort_flag, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_kv_empty(s), 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_s_free, 4);
+    mbar_init(bar_p_full, 4);
+    mbar_init(bar_o_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    *reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8) = 0;   // never raised: drain waits
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q_full, BM * D);
+      tma_load_3d(sQ, &tmQ, bar_q_full, 0, q0, bh);
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % NSTAGE, n = t / NSTAGE;
+        if (t >= NSTAGE && !mbar_wait(bar_kv_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+          break;
+        const int j0 = kv_block_at(t, T, p.kv_order) * BN;
+        mbar_arrive_expect_tx(bar_k_full(st), BN * D);
+        tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, j0, bkv);
+        mbar_arrive_expect_tx(bar_v_full(st), BN * D);
+        tma_load_3d(sV + st * BN * D, &tmV, bar_v_full(st), 0, j0, bkv);
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // drain: the last load issued into each stage must land before exit
+        const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8),
+                            p.timeout_ns};
+        for (int t = issued - 1; t >= 0 && t >= issued - NSTAGE; --t) {
+          const int st = t % NSTAGE, ph = (t / NSTAGE) & 1;
+          mbar_wait(bar_k_full(st), ph, drain, 0);
+          mbar_wait(bar_v_full(st), ph, drain, 0);
+        }
+        mbar_wait(bar_q_full, 0, drain, 0);
+      }
+    }
+  } else if (warp == 5) {
+    // ----------------------------------------------------------------- MMA --
+    constexpr uint32_t SWZ_QK = (D == 128) ? SWZ_128B : SWZ_64B;
+    constexpr uint32_t SWZ_P = (BN == 128) ? SWZ_128B : SWZ_64B;
+    constexpr uint32_t IDESC_QK = idesc_e4m3_f32(BM, BN, 0, 0);
+    constexpr uint32_t IDESC_PV = idesc_e4m3_f32(BM, D, 0, 1);
+    const uint32_t tS = tmem_base, tO = tmem_base + BN;
+    bool ok = mbar_wait(bar_q_full, 0, ctl, WAIT_MMA_Q);
+    auto issue_qk = [&](int st) {
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t a = smem_desc(sQ + 32 * kk, 16, 8 * D, SWZ_QK);
+          const uint64_t bdesc = smem_desc(sK + st * BN * D + 32 * kk, 16, 8 * D, SWZ_QK);
+          mma_e4m3_ss(tS, a, bdesc, IDESC_QK, kk > 0);
+        }
+        mma_commit(bar_s_full);
+      }
+      __syncwarp();
+    };
+    if (ok) ok = mbar_wait(bar_k_full(0), 0, ctl, WAIT_MMA_K);
+    if (ok) issue_qk(0);
+    for (int t = 0; ok && t < T; ++t) {
+      if (t + 1 < T) {
+        const int st1 = (t + 1) % NSTAGE, ph1 = ((t + 1) / NSTAGE) & 1;
+        ok = mbar_wait(bar_k_full(st1), ph1, ctl, WAIT_MMA_K) &&
+             mbar_wait(bar_s_free, t & 1, ctl, WAIT_MMA_S_FREE);
+        if (!ok) break;
+        issue_qk(st1);
+      }
+      const int st = t % NSTAGE, ph = (t / NSTAGE) & 1;
+      ok = mbar_wait(bar_v_full(st), ph, ctl, WAIT_MMA_V) &&
+           mbar_wait(bar_p_full, t & 1, ctl, WAIT_MMA_P);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 32; ++kk) {
+          const uint64_t a = smem_desc(sP + 32 * kk, 16, 8 * BN, SWZ_P);
+          const uint64_t bdesc =
+              smem_desc(sV + st * BN * D + kk * 32 * D, BN * D, 8 * D, SWZ_QK);
+          mma_e4m3_ss(tO, a, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar_o_done);
+        mma_commit(bar_kv_empty(st));
+      }
+      __syncwarp();
+    }
+    if (!ok) {
+      // drain every MMA this warp issued before TMEM is released
+      const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8), p.timeout_ns};
+      if (lane == 0) mma_commit(bar_drain);
+      __syncwarp();
+      mbar_wait(bar_drain, 0, drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax --
+    const int r = threadIdx.x;   // row within the tile; warp w reads TMEM lanes 32w..32w+31
+    const int row = q0 + r;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t tS = tmem_base + lane_off, tO = tmem_base + lane_off + BN;
+    const float c = p.scale_log2;
+    const float S = p.S;
+    float m_run = -INFINITY, l = 0.f;
+    uint32_t cnt = 0, cnt_sink = 0;
+    bool ok = true;
+    // this thread's P~ row in the swizzled tile (128B swizzle for 128-byte rows,
+    // 64B swizzle for 64-byte rows)
+    const uint32_t prow = sP + (r >> 3) * (8 * BN) + (r & 7) * BN;
+    const uint32_t pswz = (BN == 128) ? (uint32_t)(r & 7) : (uint32_t)((r & 7) >> 1);
+
+    for (int t = 0; t < T; ++t) {
+      const int j0 = kv_block_at(t, T, p.kv_order) * BN;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, t & 1, ctl, WAIT_SM_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[BN];
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc)
+        tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_s_free);
+
+      float* s = reinterpret_cast<float*>(sr);
+      const bool need_mask = (p.causal && j0 + BN - 1 > q0) || (j0 + BN > p.N);
+      if (need_mask) {
+        const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
+#pragma unroll
+        for (int j = 0; j < BN; ++j)
+          if (j0 + j > lim) s[j] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int j = 1; j < BN; ++j) mx = fmaxf(mx, s[j]);
+      const float m_new = fmaxf(m_run, mx * c);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
+      float rowsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < BN; ++j) {
+        s[j] = ex2_approx(fmaf(s[j], c, -m_use));
+        rowsum += s[j];
+      }
+      l = alpha * l + rowsum;
+      uint32_t pw[BN / 4];
+#pragma unroll
+      for (int q = 0; q < BN / 4; ++q)
+        pw[q] = pack_e4m3x4(S * s[4 * q], S * s[4 * q + 1], S * s[4 * q + 2], S * s[4 * q + 3]);
+      if constexpr (COUNT) {
+        uint32_t cblk = 0;
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          const uint32_t byte = (pw[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+          cblk += (s[j] > 0.f && byte == 0u && j0 + j >= p.n_sink) ? 1u : 0u;
+        }
+        cnt += cblk;
+        if (j0 < p.n_sink) cnt_sink += cblk;
+      }
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * cc, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(tO + 32 * cc, o);
+          }
+          tmem_wait_st();
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < BN / 16; ++q) {
+        const uint32_t dst = prow + ((q ^ pswz) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pw[4 * q]),
+                     "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full);
+      m_run = m_new;
+    }
+
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (T - 1) & 1, ctl, WAIT_EPI_O_DONE));
+    }
+    if (ok) {
+      tc_fence_after();
+      const float denom = S * l;
+      const bool live = row < p.N;
+      const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * cc, o);
+        tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), denom);
+        if (live) {
+          if constexpr (OUT_BF16) {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              uint32_t bits;
+              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(bits) : "f"(v[2 * k + 1]), "f"(v[2 * k]));
+              w[k] = bits;
+            }
+            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + obase + 32 * cc);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              out[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          } else {
+            float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.O) + obase + 32 * cc);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              out[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
+        }
+      }
+      if constexpr (COUNT) {
+        if (p.rows && live) p.rows[(size_t)bh * p.N + row] = cnt;
+        const uint32_t wsum = __reduce_add_sync(0xffffffffu, cnt);
+        const uint32_t wsink = __reduce_add_sync(0xffffffffu, cnt_sink);
+        if (lane == 0) {
+          if (wsum) atomicAdd(p.ctr, (unsigned long long)wsum);
+          if (p.ctr_sink && wsink) atomicAdd(p.ctr_sink, (unsigned long long)wsink);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag && p.status) atomicCAS(p.status, 0u, 0x100u | *abort_flag);
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------- E4M3 cast --
+__global__ void e4m3_scale_cast_kernel(const float* __restrict__ P, uint8_t* __restrict__ out,
+                                       size_t n, float S) {
+  const size_t n8 = n / 8;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const float4 a = reinterpret_cast<const float4*>(P)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(P)[2 * i + 1];
+    const uint32_t w0 = pack_e4m3x4(S * a.x, S * a.y, S * a.z, S * a.w);
+    const uint32_t w1 = pack_e4m3x4(S * b.x, S * b.y, S * b.z, S * b.w);
+    reinterpret_cast<uint2*>(out)[i] = make_uint2(w0, w1);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < n - n8 * 8) {
+    const size_t i = n8 * 8 + threadIdx.x;
+    out[i] = (uint8_t)(cvt_e4m3x2(0.f, S * P[i]) & 0xFFu);
+  }
+}
+
+}  // namespace fp8attn
+
+// ======================================================================= host
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const std::string& why) {
+  g_last_error = why;
+  return status;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D map over an E4M3 tensor [planes, rows, d] with box [d, box_rows, 1].
+bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)d * (cuuint64_t)rows};
+  cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMapSwizzle swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D, int BN, bool OUT_BF16, bool COUNT>
+cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                   const fp8attn::KParams& kp, cudaStream_t stream) {
+  using L = fp8attn::Smem<D, BN>;
+  auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 grid(kp.num_q_tiles, kp.B * kp.H);
+  kern<<<grid, fp8attn::NTHREADS, L::ALLOC, stream>>>(q, k, v, kp);
+  return cudaGetLastError();
+}
+
+template <int D, int BN>
+cudaError_t launch_dt(bool bf16, bool count, const CUtensorMap& q, const CUtensorMap& k,
+                      const CUtensorMap& v, const fp8attn::KParams& kp, cudaStream_t s) {
+  if (bf16) return count ? launch<D, BN, true, true>(q, k, v, kp, s)
+                         : launch<D, BN, true, false>(q, k, v, kp, s);
+  return count ? launch<D, BN, false, true>(q, k, v, kp, s)
+               : launch<D, BN, false, false>(q, k, v, kp, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8attn_version(void) { return 100; }
+
+size_t fp8attn_params_sizeof(void) { return sizeof(fp8attn_params); }
+
+const char* fp8attn_status_string(int status) {
+  switch (status) {
+    case FP8ATTN_OK: return "ok";
+    case FP8ATTN_EINVAL: return "invalid argument";
+    case FP8ATTN_EUNSUPPORTED: return "unsupported configuration";
+    case FP8ATTN_ECUDA: return "CUDA error";
+    case FP8ATTN_ETIMEOUT: return "bounded wait expired on the device";
+    default: return "unknown status";
+  }
+}
+
+const char* fp8attn_last_error(void) { return g_last_error.c_str(); }
+
+const char* fp8attn_device_status_string(unsigned int word) {
+  if (word == 0) return "";
+  switch (word & 0xFFu) {
+    case fp8attn::WAIT_PROD_KV_EMPTY: return "timeout: producer waiting for a free K/V stage";
+    case fp8attn::WAIT_MMA_Q: return "timeout: MMA waiting for the Q tile";
+    case fp8attn::WAIT_MMA_K: return "timeout: MMA waiting for a K tile";
+    case fp8attn::WAIT_MMA_S_FREE: return "timeout: MMA waiting for the S buffer";
+    case fp8attn::WAIT_MMA_V: return "timeout: MMA waiting for a V tile";
+    case fp8attn::WAIT_MMA_P: return "timeout: MMA waiting for the P~ tile";
+    case fp8attn::WAIT_SM_S_FULL: return "timeout: softmax waiting for S";
+    case fp8attn::WAIT_SM_O_DONE: return "timeout: softmax waiting for P~V";
+    case fp8attn::WAIT_EPI_O_DONE: return "timeout: epilogue waiting for the last P~V";
+    default: return "timeout: unknown wait";
+  }
+}
+
+int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return fail(FP8ATTN_EINVAL, "params is NULL");
+  if (p->B < 0 || p->H < 0 || p->N < 0) return fail(FP8ATTN_EINVAL, "B, H, N must be >= 0");
+  if (p->H_kv <= 0 && p->H > 0) return fail(FP8ATTN_EINVAL, "H_kv must be >= 1");
+  if (p->H > 0 && p->H % p->H_kv) return fail(FP8ATTN_EINVAL, "H must be a multiple of H_kv");
+  if (p->d != 64 && p->d != 128) return fail(FP8ATTN_EUNSUPPORTED, "d must be 64 or 128");
+  const int bn = p->block_n == 0 ? 128 : p->block_n;
+  if (bn != 64 && bn != 128) return fail(FP8ATTN_EUNSUPPORTED, "block_n must be 0, 64 or 128");
+  if (p->causal != 0 && p->causal != 1) return fail(FP8ATTN_EINVAL, "causal must be 0 or 1");
+  if (!std::isfinite(p->scale) || !(p->scale > 0.f))
+    return fail(FP8ATTN_EINVAL, "scale must be finite and > 0");
+  if (!std::isfinite(p->S) || !(p->S > 0.f)) return fail(FP8ATTN_EINVAL, "S must be finite and > 0");
+  if (p->kv_order != FP8ATTN_KV_FORWARD && p->kv_order != FP8ATTN_KV_REVERSE)
+    return fail(FP8ATTN_EINVAL, "kv_order must be 0 (forward) or 1 (reverse)");
+  if (p->n_sink < 0 || p->n_sink > p->N) return fail(FP8ATTN_EINVAL, "n_sink must be in [0, N]");
+  if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
+    return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
+  if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
+    return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
+  if ((long long)p->B * p->H > 65535LL * 65535LL) return fail(FP8ATTN_EINVAL, "B*H too large");
+  if ((long long)p->B * p->H * p->N == 0) return FP8ATTN_OK;   // nothing to compute
+  if (!p->Q || !p->K || !p->V || !p->O) return fail(FP8ATTN_EINVAL, "Q, K, V, O must be non-NULL");
+  if (!aligned16(p->Q) || !aligned16(p->K) || !aligned16(p->V) || !aligned16(p->O))
+    return fail(FP8ATTN_EINVAL, "Q, K, V, O must be 16-byte aligned");
+  if ((p->collapse_ctr && ((uintptr_t)p->collapse_ctr & 7)) ||
+      (p->collapse_sink_ctr && ((uintptr_t)p->collapse_sink_ctr & 7)) ||
+      (p->collapse_rows && ((uintptr_t)p->collapse_rows & 3)) ||
+      (p->status_word && ((uintptr_t)p->status_word & 3)))
+    return fail(FP8ATTN_EINVAL, "counter / status pointers must be naturally aligned");
+
+  CUtensorMap mq, mk, mv;
+  if (!encode_fn()) return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled is not available");
+  if (!make_map(&mq, p->Q, p->d, p->N, p->B * p->H, fp8attn::BM) ||
+      !make_map(&mk, p->K, p->d, p->N, p->B * p->H_kv, bn) ||
+      !make_map(&mv, p->V, p->d, p->N, p->B * p->H_kv, bn))
+    return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled failed");
+
+  fp8attn::KParams kp;
+  kp.B = p->B;
+  kp.H = p->H;
+  kp.Hkv = p->H_kv;
+  kp.N = p->N;
+  kp.group = p->H / p->H_kv;
+  kp.causal = p->causal;
+  kp.kv_order = p->kv_order;
+  kp.n_sink = p->n_sink;
+  kp.num_q_tiles = (p->N + fp8attn::BM - 1) / fp8attn::BM;
+  kp.scale_log2 = p->scale * fp8attn::LOG2E;
+  kp.S = p->S;
+  kp.O = p->O;
+  kp.ctr = p->collapse_ctr;
+  kp.ctr_sink = p->collapse_sink_ctr;
+  kp.rows = p->collapse_rows;
+  kp.status = p->status_word;
+  kp.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
+  if (kp.B * kp.H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
+
+  const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;
+  const bool count = p->collapse_ctr != nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (p->d == 128)
+    e = (bn == 128) ? launch_dt<128, 128>(bf16, count, mq, mk, mv, kp, s)
+                    : launch_dt<128, 64>(bf16, count, mq, mk, mv, kp, s);
+  else
+    e = (bn == 128) ? launch_dt<64, 128>(bf16, count, mq, mk, mv, kp, s)
+                    : launch_dt<64, 64>(bf16, count, mq, mk, mv, kp, s);
+  if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return FP8ATTN_OK;
+}
+
+int fp8_attn_fwd(const void* Q, const void* K, const void* V, void* O, int B, int H, int N, int d,
+                 int causal, float scale, float S, int kv_order, int n_sink,
+                 unsigned long long* collapse_ctr, fp8attn_stream_t stream) {
+  fp8attn_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.O = O;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H;
+  p.N = N;
+  p.d = d;
+  p.causal = causal;
+  p.scale = scale;
+  p.S = S;
+  p.kv_order = kv_order;
+  p.n_sink = n_sink;
+  p.o_dtype = FP8ATTN_O_BF16;
+  p.block_n = 128;
+  p.collapse_ctr = collapse_ctr;
+  return fp8_attn_fwd_ex(&p, stream);
+}
+
+int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
+                        fp8attn_stream_t stream) {
+  g_last_error.clear();
+  if (n == 0) return FP8ATTN_OK;
+  if (!P || !out) return fail(FP8ATTN_EINVAL, "P and out must be non-NULL");
+  if (!aligned16(P) || !aligned16(out)) return fail(FP8ATTN_EINVAL, "P and out must be 16-byte aligned");
+  if (!std::isfinite(S)) return fail(FP8ATTN_EINVAL, "S must be finite");
+  const size_t n8 = n / 8;
+  int blocks = (int)std::min<size_t>((n8 + 255) / 256, (size_t)148 * 16);
+  if (blocks < 1) blocks = 1;
+  fp8attn::e4m3_scale_cast_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      P, out, n, S);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return FP8ATTN_OK;
+}
+
+}  // extern "C"

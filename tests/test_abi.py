@@ -1,0 +1,96 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched): the
+library builds for sm_100a and loads, exports every entry point that
+include/fp8attn.h declares, agrees on the parameter-struct layout, and
+rejects invalid arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from online_softmax_tcgen05_b200 import _binding
+from online_softmax_tcgen05_b200._binding import EINVAL, EUNSUPPORTED, OK, Params
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "fp8attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    pat = r"^\s*(?:const\s+)?(?:unsigned\s+)?(?:int|char|size_t|void|float)\s*\**\s*(\w+)\s*\("
+    return sorted(set(re.findall(pat, text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _binding.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "fp8_attn_fwd" in names and "fp8_attn_fwd_ex" in names and "fp8_e4m3_scale_cast" in names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _binding.SIGNATURES, n
+
+
+def test_params_layout(lib):
+    assert lib.fp8attn_params_sizeof() == ctypes.sizeof(Params)
+    assert lib.fp8attn_version() == 100
+
+
+def test_status_strings(lib):
+    for s in (0, -1, -2, -3, -4):
+        assert _binding.status_string(s)
+    assert _binding.device_status_string(0) == ""
+    assert "timeout" in _binding.device_status_string(0x107)
+
+
+FAKE = 0x10000   # never dereferenced: every case below fails validation first
+
+
+def base_params(**kw):
+    p = dict(Q=FAKE, K=FAKE, V=FAKE, O=FAKE, B=1, H=2, H_kv=1, N=256, d=128, causal=0,
+             scale=0.088, S=256.0, kv_order=1, n_sink=4, o_dtype=0, block_n=0,
+             collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None, status_word=None,
+             timeout_ns=0)
+    p.update(kw)
+    return Params(**p)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), EUNSUPPORTED), (dict(d=256), EUNSUPPORTED), (dict(block_n=32), EUNSUPPORTED),
+    (dict(H=3, H_kv=2), EINVAL), (dict(H_kv=0), EINVAL), (dict(N=-1), EINVAL),
+    (dict(S=0.0), EINVAL), (dict(S=-1.0), EINVAL), (dict(S=float("nan")), EINVAL),
+    (dict(S=float("inf")), EINVAL), (dict(scale=float("nan")), EINVAL), (dict(scale=0.0), EINVAL),
+    (dict(kv_order=2), EINVAL), (dict(causal=2), EINVAL), (dict(n_sink=-1), EINVAL),
+    (dict(n_sink=257), EINVAL), (dict(o_dtype=5), EINVAL), (dict(Q=None), EINVAL),
+    (dict(O=FAKE + 8), EINVAL), (dict(K=FAKE + 1), EINVAL),
+    (dict(collapse_rows=FAKE), EINVAL), (dict(collapse_ctr=FAKE + 4), EINVAL),
+])
+def test_invalid_arguments_rejected_before_launch(lib, kw, status):
+    p = base_params(**kw)
+    assert lib.fp8_attn_fwd_ex(ctypes.byref(p), None) == status
+    assert _binding.last_error() != ""
+
+
+def test_empty_problem_is_a_noop(lib):
+    for kw in (dict(B=0), dict(H=0), dict(N=0, n_sink=0)):
+        p = base_params(Q=None, K=None, V=None, O=None, **kw)
+        assert lib.fp8_attn_fwd_ex(ctypes.byref(p), None) == OK
+
+
+def test_null_params_and_short_form_validation(lib):
+    assert lib.fp8_attn_fwd_ex(None, None) == EINVAL
+    assert lib.fp8_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, 0, 0.1, 256.0, 0, 0, None,
+                            None) == EUNSUPPORTED
+    assert lib.fp8_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, 0.1, 256.0, 3, 0, None,
+                            None) == EINVAL
+
+
+def test_cast_validation(lib):
+    assert lib.fp8_e4m3_scale_cast(None, None, 0, 1.0, None) == OK
+    assert lib.fp8_e4m3_scale_cast(None, FAKE, 16, 1.0, None) == EINVAL
+    assert lib.fp8_e4m3_scale_cast(FAKE, FAKE, 16, float("nan"), None) == EINVAL
+    assert lib.fp8_e4m3_scale_cast(FAKE + 4, FAKE, 16, 1.0, None) == EINVAL
