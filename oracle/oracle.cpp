@@ -23,6 +23,7 @@
 // All FP32 sums run left to right in the order stated at each loop.
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <limits>
 #include <vector>
@@ -216,7 +217,9 @@ int oracle_attn_exact(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
 // Per query row (FP32 throughout):
 //   m = -inf, l = 0, acc = 0
 //   for each KV block in the visiting order (forward: 0..last, reverse: last..0;
-//   last = floor(i / block_n) when causal, else N/block_n - 1):
+//   last = floor(i / block_n) when causal, else ceil(N / block_n) - 1; when
+//   block_n does not divide N the last block holds the remaining N mod block_n
+//   keys):
 //     s_j    = fl32(scale * fl32(sum_k q_k k_jk))   (k ascending), -inf if j > i (causal)
 //     m'     = max(m, max_j s_j)
 //     alpha  = exp(m - m')    (0 when m = -inf; 1 when m' = -inf)
@@ -236,12 +239,12 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
                         const int64_t* rows, int64_t nrows,
                         float* O, uint32_t* collapse_rows, uint64_t* collapse_totals,
                         int nthreads) {
-    if (H % Hkv || block_n <= 0 || N % block_n) return -1;
+    if (H % Hkv || block_n <= 0) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
     if (nthreads > 0) omp_set_num_threads(nthreads);
     const int group = H / Hkv;
-    const int nblocks = N / block_n;
+    const int nblocks = (N + block_n - 1) / block_n;
     uint64_t tot_sink = 0, tot_other = 0;
     #pragma omp parallel reduction(+ : tot_sink, tot_other)
     {
@@ -262,7 +265,8 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
             for (int step = 0; step <= last; ++step) {
                 const int blk = (kv_order == 0) ? step : last - step;
                 const int j0 = blk * block_n;
-                for (int jj = 0; jj < block_n; ++jj) {
+                const int nb = std::min(block_n, N - j0);   // keys in this block
+                for (int jj = 0; jj < nb; ++jj) {
                     int j = j0 + jj;
                     if (causal && j > i) { s[jj] = kNegInf; continue; }
                     const uint8_t* kp = K + kvbase + (int64_t)j * d;
@@ -271,12 +275,12 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
                     s[jj] = scale * dot;
                 }
                 float alpha;
-                int c = softmax_block(s.data(), block_n, j0, n_sink, S, st, pt.data(), &alpha);
+                int c = softmax_block(s.data(), nb, j0, n_sink, S, st, pt.data(), &alpha);
                 row_collapse += (uint32_t)c;
                 if (block_has_sink(blk, block_n, n_sink)) tot_sink += (uint64_t)c;
                 else tot_other += (uint64_t)c;
                 for (int k = 0; k < d; ++k) acc[k] = alpha * acc[k];
-                for (int jj = 0; jj < block_n; ++jj) {
+                for (int jj = 0; jj < nb; ++jj) {
                     float pv = g_dec[pt[jj]];
                     if (pv == 0.0f) continue;   // adds exactly +0 (v is finite)
                     const uint8_t* vp = V + kvbase + (int64_t)(j0 + jj) * d;
@@ -304,9 +308,9 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
 int oracle_collapse_logits(const float* logits, int64_t nrows, int N, int block_n, int n_sink,
                            float S, int kv_order, uint32_t* collapse_rows,
                            uint64_t* collapse_totals, int nthreads) {
-    if (block_n <= 0 || N % block_n) return -1;
+    if (block_n <= 0) return -1;
     if (nthreads > 0) omp_set_num_threads(nthreads);
-    const int nblocks = N / block_n;
+    const int nblocks = (N + block_n - 1) / block_n;
     uint64_t tot_sink = 0, tot_other = 0;
     #pragma omp parallel reduction(+ : tot_sink, tot_other)
     {
@@ -318,7 +322,8 @@ int oracle_collapse_logits(const float* logits, int64_t nrows, int N, int block_
             for (int step = 0; step < nblocks; ++step) {
                 int blk = (kv_order == 0) ? step : nblocks - 1 - step;
                 float alpha;
-                int c = softmax_block(logits + r * (int64_t)N + (int64_t)blk * block_n, block_n,
+                int nb = std::min(block_n, N - blk * block_n);
+                int c = softmax_block(logits + r * (int64_t)N + (int64_t)blk * block_n, nb,
                                       blk * block_n, n_sink, S, st, pt.data(), &alpha);
                 rc += (uint32_t)c;
                 if (block_has_sink(blk, block_n, n_sink)) tot_sink += (uint64_t)c;

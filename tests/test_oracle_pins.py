@@ -258,7 +258,7 @@ def brute_force_rows(oracle_mod, Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, 
                 prods = (q[b, h, i][None, :] * k[b, h // g]).astype(np.float32)
                 dots = np.cumsum(prods, axis=1, dtype=np.float32)[:, -1]
                 s = (np.float32(scale) * dots).astype(np.float32)
-                last = i // block_n if causal else N // block_n - 1
+                last = i // block_n if causal else (N + block_n - 1) // block_n - 1
                 blocks = list(range(last + 1))
                 if order == 1:
                     blocks = blocks[::-1]
@@ -290,7 +290,8 @@ def brute_force_rows(oracle_mod, Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, 
 
 @pytest.mark.parametrize("N,d,block_n,causal", [(64, 16, 16, 0), (128, 16, 32, 1),
                                                 (256, 64, 64, 0), (256, 64, 64, 1),
-                                                (192, 32, 32, 1)])
+                                                (192, 32, 32, 1), (200, 32, 64, 0),
+                                                (200, 32, 64, 1), (77, 16, 32, 1)])
 def test_emulation_matches_brute_force(oracle_mod, N, d, block_n, causal):
     B, H, Hkv = 1, 2, 1
     W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 9.0, seed=16 + N + d)
