@@ -1,0 +1,364 @@
+"""Benchmark of the FP8 attention forward with P-cast scale S and KV order.
+
+Workload (one step): the causal GQA prefill of the P-cast study's LLM shape,
+B=1, H=32 query heads over H_kv=8 KV heads, N=32768, d=128, E4M3 Q/K/V from
+the seeded sink construction (n_sink=4, Delta=8), S=256, reverse KV order,
+O in BF16, collapse counter on: one launch of the library's tcgen05 kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  value = algorithmic TFLOP/s of the whole job
+(2*B*H*N^2*d per causal step, all ranks' work / the slowest rank's time);
+e2e = the same metric through the public API with pinned host buffers,
+host<->device copies inside the timed region; roofline = the kernel's
+achieved TFLOP/s against the FP8 dense peak (measured BF16 GEMM x 2);
+cpu_baseline = the CPU oracle on a bounded sample of the same rows.
+Multi-GPU (torchrun): every rank runs its own independent prefill (weak
+scaling); no collective is on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+CFG = dict(B=1, H=32, H_kv=8, N=32768, d=128, causal=1, S=256.0, kv_order=1, n_sink=4,
+           delta=8.0, block_n=128)
+WORKLOAD = ("causal GQA prefill B=1 H=32/H_kv=8 N=32768 d=128 E4M3, sink construction "
+            "n_sink=4 Delta=8, S=256, reverse KV order, O bf16, collapse counter on")
+METRIC = "FP8 attn fwd TFLOPS & % of B200 FP8 peak; P-collapse rate vs F(Δ,S)"
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def algorithmic_flops(B, H, N, d, causal):
+    return (2 if causal else 4) * B * H * N * N * d
+
+
+def peak_tflops():
+    """FP8 dense peak: the measured BF16 GEMM burst peak x 2 (nominal fp8/bf16
+    ratio), else the machine's fallback figure."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return 2.0 * float(pk["bf16_tflops"]), "measured bf16 burst x 2 (MEASURED_PEAKS.json)"
+    except Exception:
+        return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2"
+
+
+def smi_index(local_rank):
+    """nvidia-smi index of this process's GPU (CUDA_VISIBLE_DEVICES aware)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in vis.split(",") if x.strip()]
+    if local_rank < len(ids) and ids[local_rank].isdigit():
+        return int(ids[local_rank])
+    return local_rank
+
+
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) during the timed region."""
+
+    def __init__(self, index):
+        self.index = smi_index(index)
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + CLOCK_FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def make_inputs(seed, dev):
+    import torch
+    import workload
+    from online_softmax_tcgen05_b200 import e4m3_cast
+    W = workload.make_sink_workload(CFG["B"], CFG["H"], CFG["H_kv"], CFG["N"], CFG["d"],
+                                    CFG["n_sink"], CFG["delta"], seed=seed)
+    qkv = [e4m3_cast(torch.from_numpy(x).to(dev)) for x in (W.q, W.k, W.v)]
+    return W, qkv
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import online_softmax_tcgen05_b200 as fa
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    fa.load_library()
+    import workload
+    W, (q, k, v) = make_inputs(workload.CONFIG_SEED_BASE + 3 + 1000 * rank, dev)
+    B, H, Hkv, N, d = CFG["B"], CFG["H"], CFG["H_kv"], CFG["N"], CFG["d"]
+    scale = 1.0 / math.sqrt(d)
+    O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    ctr = torch.zeros(2, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(count=True):
+        fa.fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=Hkv, N=N, d=d, causal=True, scale=scale,
+                           S=CFG["S"], kv_order=CFG["kv_order"], n_sink=CFG["n_sink"],
+                           o_dtype=fa.O_BF16, block_n=CFG["block_n"],
+                           collapse_ctr=ctr[0:1] if count else None,
+                           collapse_sink_ctr=ctr[1:2] if count else None, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, steps):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for _ in range(args.warmup):
+        step(True)
+        step(False)
+    torch.cuda.synchronize()
+    ctr.zero_()
+    with ClockSampler(local_rank) as clk:
+        ms_on = timed(lambda: step(True), args.steps)
+    collapse_total, collapse_sink = (int(x) for x in ctr.cpu().tolist())
+    ms_off = timed(lambda: step(False), args.steps)
+
+    flops = algorithmic_flops(B, H, N, d, True)
+    step_ms = ms_on / args.steps
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    kernel_tflops = flops / (step_ms * 1e-3) / 1e12
+    peak, peak_src = peak_tflops()
+
+    if args.mode == "kernel":
+        if rank != 0:
+            return None
+        return {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+                "mode": "kernel only", "value_counter_off":
+                round(world * flops / (ms_off / args.steps * 1e-3) / 1e12, 2)}
+
+    # end to end through the public API: pinned host E4M3 inputs -> device ->
+    # kernel -> BF16 output back to pinned host memory, every step
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+
+    def e2e_step():
+        fa.attention(qh, kh, vh, causal=True, scale=scale, S=CFG["S"], kv_order=CFG["kv_order"],
+                     n_sink=CFG["n_sink"], block_n=CFG["block_n"], count_collapse=True, out=oh)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    e2e_steps = max(2, args.steps // 2)
+    ms_e2e = timed(e2e_step, e2e_steps)
+    e2e_value = world * flops / (ms_e2e / e2e_steps * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + 16
+
+    if world > 1:
+        ct = torch.tensor([collapse_total, collapse_sink], dtype=torch.int64, device=dev)
+        dist.all_reduce(ct)
+        collapse_total, collapse_sink = (int(x) for x in ct.tolist())
+
+    if rank != 0:
+        return None
+    import oracle
+    pairs = world * B * H * (N - CFG["n_sink"]) * (N - CFG["n_sink"] + 1) // 2
+    frac = collapse_total / args.steps / pairs
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, **CFG, "per_rank": "independent prefill per GPU",
+                   "l2": "inputs 201 MB > 126 MB L2, no flush"},
+        "value_counter_off": round(world * flops / (ms_off / args.steps * 1e-3) / 1e12, 2),
+        "pct_of_fp8_peak": {"measured": round(kernel_tflops / peak, 4),
+                            "nominal_4500": round(kernel_tflops / 4500.0, 4)},
+        "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2),
+                     "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(kernel_tflops / peak, 4), "traffic": None,
+                     "peak_source": peak_src + " (of measured)" if "measured" in peak_src
+                     else peak_src},
+        "collapse": {"fraction": frac, "count_per_step": collapse_total // args.steps // world,
+                     "in_sink_block": collapse_sink // args.steps // world,
+                     "closed_form_forward_F": oracle.underflow_fraction_closed(CFG["delta"],
+                                                                               CFG["S"])},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / e2e_steps, 3)},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(W, seconds_hint=True)
+    return line
+
+
+def sample_rows(n_rows, seed=7):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    total = CFG["B"] * CFG["H"] * CFG["N"]
+    return np.sort(rng.choice(total, n_rows, replace=False)).astype(np.int64)
+
+
+def oracle_sample(W, rows, Q8=None, K8=None, V8=None):
+    """Time the oracle's FP8 emulation on the given rows of the workload;
+    returns (seconds, algorithmic FLOPs of those rows)."""
+    import oracle
+    N, d = CFG["N"], CFG["d"]
+    if Q8 is None:
+        Q8, K8, V8 = (oracle.e4m3_encode(x) for x in (W.q, W.k, W.v))
+    t0 = time.perf_counter()
+    oracle.attn_emulate(Q8, K8, V8, CFG["B"], CFG["H"], CFG["H_kv"], N, d, 1,
+                        1.0 / math.sqrt(d), CFG["S"], CFG["kv_order"], CFG["block_n"],
+                        CFG["n_sink"], o_bf16=True, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = float(sum(4 * d * ((int(r) % N) + 1) for r in rows))
+    return dt, flops, (Q8, K8, V8)
+
+
+def cpu_baseline(W, seconds_hint=True, n_rows=32768):
+    rows = sample_rows(n_rows)
+    dt, flops, _ = oracle_sample(W, rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": "%d seeded random query rows of the %d (all heads and positions), "
+                      "FP8 pipeline emulation, %.1f s" % (n_rows, CFG["B"] * CFG["H"] * CFG["N"],
+                                                          dt)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm, on rank 0 only."""
+    if rank != 0:
+        return None
+    import workload
+    W = workload.make_sink_workload(CFG["B"], CFG["H"], CFG["H_kv"], CFG["N"], CFG["d"],
+                                    CFG["n_sink"], CFG["delta"],
+                                    seed=workload.CONFIG_SEED_BASE + 3)
+    rows_per_step = 1024
+    enc = None
+    for i in range(args.warmup):
+        _, _, enc = oracle_sample(W, sample_rows(rows_per_step, seed=100 + i),
+                                  *(enc or (None, None, None)))
+    tot_t, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl, enc = oracle_sample(W, sample_rows(rows_per_step, seed=200 + i),
+                                    *(enc or (None, None, None)))
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = ("%d seeded random query rows per step of the %d, FP8 pipeline emulation"
+              % (rows_per_step, CFG["B"] * CFG["H"] * CFG["N"]))
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": WORKLOAD, **CFG}, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["full", "kernel"], default="full",
+                    help="kernel: only the device-timed kernel loop (for profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            sys.exit("run multi-GPU through torchrun: --nproc-per-node %d" % args.gpus)
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    pg = False
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+        pg = True
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

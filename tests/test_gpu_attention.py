@@ -257,5 +257,19 @@ def test_long_context_full_size():
     rows = _boundary_rows(B, H, N, 8)
     _, tot, sink_tot, _ = check_case(W, ins, 1, 256.0, 1, 128, f32=False, rows=rows,
                                      what="long rev 256")
-    assert tot == sink_tot
+    # Reverse + 256 leaves (almost) nothing outside the sink block.  The paper's
+    # < 1e-12 bound is for unit-variance logits; here the per-row logit spread
+    # varies with |g_i|, so at N = 131072 a few far-tail entries can underflow.
+    # With n_sink = block_n only entries outside the sink block are counted (the
+    # arithmetic is unchanged): the rows holding them must agree with the oracle.
+    pairs = H * N * (N + 1) // 2
+    assert (tot - sink_tot) / pairs < 1e-9
+    _, out_tot, _, out_rows = run_gpu(ins, B, H, Hkv, N, d, 1, 256.0, 1, 128, 128, f32=False)
+    assert out_tot == tot - sink_tot
+    hit = np.flatnonzero(out_rows)
+    if hit.size:
+        (_, Q8), (_, K8), (_, V8) = ins
+        _, cr, _ = oracle.attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, 1, W.scale, 256.0, 1, 128,
+                                       128, o_bf16=True, rows=hit)
+        assert np.abs(cr.astype(np.int64) - out_rows[hit]).sum() <= 1, (hit, cr, out_rows[hit])
     check_case(W, ins, 1, 1.0, 0, 128, f32=False, rows=rows[::3], what="long fwd 1")
