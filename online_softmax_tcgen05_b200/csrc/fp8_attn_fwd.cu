@@ -275,36 +275,76 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
       float* s = reinterpret_cast<float*>(sr);
       const bool need_mask = (p.causal && j0 + BN - 1 > q0) || (j0 + BN > p.N);
+      const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
       if (need_mask) {
-        const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
 #pragma unroll
         for (int j = 0; j < BN; ++j)
           if (j0 + j > lim) s[j] = -INFINITY;
       }
-      float mx = s[0];
+      // row max: 16 independent chains, then a tree
+      float mx16[16];
 #pragma unroll
-      for (int j = 1; j < BN; ++j) mx = fmaxf(mx, s[j]);
-      const float m_new = fmaxf(m_run, mx * c);
+      for (int i = 0; i < 16; ++i) mx16[i] = s[i];
+#pragma unroll
+      for (int j = 16; j < BN; ++j) mx16[j & 15] = fmaxf(mx16[j & 15], s[j]);
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + w]);
+      const float m_new = fmaxf(m_run, mx16[0] * c);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-      float rowsum = 0.f;
+      // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+      float2 acc8[8];
 #pragma unroll
-      for (int j = 0; j < BN; ++j) {
-        s[j] = ex2_approx(fmaf(s[j], c, -m_use));
-        rowsum += s[j];
+      for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < BN / 2; ++q) {
+        const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
+        s[2 * q] = ex2_approx(y.x);
+        s[2 * q + 1] = ex2_approx(y.y);
+        acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
       }
-      l = alpha * l + rowsum;
+#pragma unroll
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
+      l = alpha * l + (acc8[0].x + acc8[0].y);
+      // S * p (packed FMUL2), then the E4M3 cast, four keys per word
+      const float2 S2 = make_float2(S, S);
       uint32_t pw[BN / 4];
 #pragma unroll
-      for (int q = 0; q < BN / 4; ++q)
-        pw[q] = pack_e4m3x4(S * s[4 * q], S * s[4 * q + 1], S * s[4 * q + 2], S * s[4 * q + 3]);
+      for (int q = 0; q < BN / 4; ++q) {
+        const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
+        const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
+        pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
+      }
       if constexpr (COUNT) {
-        uint32_t cblk = 0;
+        // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
+        // negative, so byte 0 <=> the cast flushed S*p to zero.  Zero bytes are
+        // found four at a time; blocks that hold a sink or a masked key restrict
+        // the count to the lanes with n_sink <= j <= last visible key.
+        uint32_t zacc = 0;
+        if (j0 >= p.n_sink && !need_mask) {
 #pragma unroll
-        for (int j = 0; j < BN; ++j) {
-          const uint32_t byte = (pw[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-          cblk += (s[j] > 0.f && byte == 0u && j0 + j >= p.n_sink) ? 1u : 0u;
+          for (int q = 0; q < BN / 4; ++q) {
+            const uint32_t w = pw[q];
+            zacc += ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu) >> 7;
+          }
+        } else {
+          const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);   // block-local
+#pragma unroll
+          for (int q = 0; q < BN / 4; ++q) {
+            const uint32_t w = pw[q];
+            uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
+            const int a = lo - 4 * q, bq = hi - 4 * q;   // lanes a..bq of this word are valid
+            const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
+            const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
+            zacc += (y & mlo & mhi) >> 7;
+          }
         }
+        const uint32_t cblk = (zacc * 0x01010101u) >> 24;   // byte lanes hold <= BN/4 each
         cnt += cblk;
         if (j0 < p.n_sink) cnt_sink += cblk;
       }
@@ -318,8 +358,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             uint32_t o[32];
             tmem_ld32(tO + 32 * cc, o);
             tmem_wait_ld();
+            const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            for (int k = 0; k < 32; k += 2) {
+              const float2 r2 = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), a2);
+              o[k] = __float_as_uint(r2.x);
+              o[k + 1] = __float_as_uint(r2.y);
+            }
             tmem_st32(tO + 32 * cc, o);
           }
           tmem_wait_st();
@@ -377,6 +422,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       if constexpr (COUNT) {
+        if (!live) cnt = cnt_sink = 0;   // padding rows past a ragged N
         if (p.rows && live) p.rows[(size_t)bh * p.N + row] = cnt;
         const uint32_t wsum = __reduce_add_sync(0xffffffffu, cnt);
         const uint32_t wsink = __reduce_add_sync(0xffffffffu, cnt_sink);
