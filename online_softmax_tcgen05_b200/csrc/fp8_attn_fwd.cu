@@ -37,6 +37,7 @@
 #include <string>
 
 #include "fp8attn.h"
+#include "exp2_poly.cuh"
 #include "sm100.cuh"
 
 namespace fp8attn {
@@ -45,6 +46,13 @@ constexpr int BM = 128;         // query rows per CTA (= MMA M, = TMEM lanes)
 constexpr int NSTAGE = 2;       // K/V ring depth
 constexpr int NTHREADS = 192;   // 4 softmax warps + TMA warp + MMA warp
 constexpr float LOG2E = 1.4426950408889634f;
+// Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
+// (exp2_poly.cuh) and the rest on MUFU ex2: the two units then share the
+// exponentials of the softmax.
+#ifndef FP8ATTN_POLY_OF_8
+#define FP8ATTN_POLY_OF_8 2
+#endif
+constexpr int POLY_OF_8 = FP8ATTN_POLY_OF_8;
 
 // device status codes (status_word): 0x100 | where the wait gave up
 enum : uint32_t {
@@ -80,8 +88,9 @@ struct Smem {
   static constexpr int V = K + NSTAGE * BN * D;
   static constexpr int P = V + NSTAGE * BN * D;
   static constexpr int BAR = P + BM * BN;
-  // barriers: q_full, k_full[2], v_full[2], kv_empty[2], s_full, s_free, p_full, o_done, drain
-  static constexpr int NBAR = 1 + 3 * NSTAGE + 5;
+  // barriers: q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full, s_free, p_full,
+  // o_done, drain
+  static constexpr int NBAR = 1 + 4 * NSTAGE + 5;
   static constexpr int MISC = BAR + 8 * NBAR;   // tmem base slot, abort flag
   static constexpr int BYTES = MISC + 16;
   // slack to align the base to 1024, and at least 80 KB so that no more than two
@@ -109,8 +118,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t bar_q_full = bar0;
   auto bar_k_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
-  auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
-  const uint32_t bar_s_full = bar0 + 8u * (1 + 3 * NSTAGE);
+  auto bar_k_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
+  auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
+  const uint32_t bar_s_full = bar0 + 8u * (1 + 4 * NSTAGE);
   const uint32_t bar_s_free = bar_s_full + 8;
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_o_done = bar_s_full + 24;
@@ -133,7 +143,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(bar_k_full(s), 1);
       mbar_init(bar_v_full(s), 1);
-      mbar_init(bar_kv_empty(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+      mbar_init(bar_v_empty(s), 1);
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_s_free, 4);
@@ -163,27 +174,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q_full, BM * D);
       tma_load_3d(sQ, &tmQ, bar_q_full, 0, q0, bh);
-      int issued = 0;
-      for (int t = 0; t < T; ++t) {
+      // K runs one KV step ahead of V: K(t+1) needs only QK^T(t-1) to have
+      // released its stage, V(t) needs P~V(t-2).
+      int k_issued = 0, v_issued = 0;
+      auto load_k = [&](int t) -> bool {
         const int st = t % NSTAGE, n = t / NSTAGE;
-        if (t >= NSTAGE && !mbar_wait(bar_kv_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
-          break;
-        const int j0 = kv_block_at(t, T, p.kv_order) * BN;
+        if (t >= NSTAGE && !mbar_wait(bar_k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+          return false;
         mbar_arrive_expect_tx(bar_k_full(st), BN * D);
-        tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, j0, bkv);
+        tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
+                    bkv);
+        k_issued = t + 1;
+        return true;
+      };
+      bool ok = load_k(0);
+      for (int t = 0; ok && t < T; ++t) {
+        if (t + 1 < T && !load_k(t + 1)) break;
+        const int st = t % NSTAGE, n = t / NSTAGE;
+        if (t >= NSTAGE && !mbar_wait(bar_v_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+          break;
         mbar_arrive_expect_tx(bar_v_full(st), BN * D);
-        tma_load_3d(sV + st * BN * D, &tmV, bar_v_full(st), 0, j0, bkv);
-        issued = t + 1;
+        tma_load_3d(sV + st * BN * D, &tmV, bar_v_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
+                    bkv);
+        v_issued = t + 1;
       }
       if (*abort_flag) {
         // drain: the last load issued into each stage must land before exit
         const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8),
                             p.timeout_ns};
-        for (int t = issued - 1; t >= 0 && t >= issued - NSTAGE; --t) {
-          const int st = t % NSTAGE, ph = (t / NSTAGE) & 1;
-          mbar_wait(bar_k_full(st), ph, drain, 0);
-          mbar_wait(bar_v_full(st), ph, drain, 0);
-        }
+        for (int t = k_issued - 1; t >= 0 && t >= k_issued - NSTAGE; --t)
+          mbar_wait(bar_k_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
+        for (int t = v_issued - 1; t >= 0 && t >= v_issued - NSTAGE; --t)
+          mbar_wait(bar_v_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
         mbar_wait(bar_q_full, 0, drain, 0);
       }
     }
@@ -205,6 +227,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mma_e4m3_ss(tS, a, bdesc, IDESC_QK, kk > 0);
         }
         mma_commit(bar_s_full);
+        mma_commit(bar_k_empty(st));
       }
       __syncwarp();
     };
@@ -232,7 +255,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mma_e4m3_ss(tO, a, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar_o_done);
-        mma_commit(bar_kv_empty(st));
+        mma_commit(bar_v_empty(st));
       }
       __syncwarp();
     }
@@ -302,8 +325,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
       for (int q = 0; q < BN / 2; ++q) {
         const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
-        s[2 * q] = ex2_approx(y.x);
-        s[2 * q + 1] = ex2_approx(y.y);
+        if ((q & 7) < POLY_OF_8) {
+          const float2 e = exp2_poly2(y);
+          s[2 * q] = e.x;
+          s[2 * q + 1] = e.y;
+        } else {
+          s[2 * q] = ex2_approx(y.x);
+          s[2 * q + 1] = ex2_approx(y.y);
+        }
         acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
       }
 #pragma unroll
@@ -349,26 +378,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (j0 < p.n_sink) cnt_sink += cblk;
       }
       if (t > 0) {
+        // P~V(t-1) must be done: it reads the P~ tile and accumulates into O
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * cc, o);
-            tmem_wait_ld();
-            const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const float2 r2 = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), a2);
-              o[k] = __float_as_uint(r2.x);
-              o[k + 1] = __float_as_uint(r2.y);
-            }
-            tmem_st32(tO + 32 * cc, o);
-          }
-          tmem_wait_st();
-        }
       }
 #pragma unroll
       for (int q = 0; q < BN / 16; ++q) {
@@ -376,6 +389,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pw[4 * q]),
                      "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
                      : "memory");
+      }
+      if (t > 0) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          // O *= alpha for this warp's 32 rows, 64 TMEM columns per round trip
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; cc += 2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tO + 32 * cc, o0);
+            tmem_ld32(tO + 32 * cc + 32, o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              float2 r0 = __fmul2_rn(make_float2(__uint_as_float(o0[k]), __uint_as_float(o0[k + 1])), a2);
+              float2 r1 = __fmul2_rn(make_float2(__uint_as_float(o1[k]), __uint_as_float(o1[k + 1])), a2);
+              o0[k] = __float_as_uint(r0.x);
+              o0[k + 1] = __float_as_uint(r0.y);
+              o1[k] = __float_as_uint(r1.x);
+              o1[k + 1] = __float_as_uint(r1.y);
+            }
+            tmem_st32(tO + 32 * cc, o0);
+            tmem_st32(tO + 32 * cc + 32, o1);
+          }
+          tmem_wait_st();
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
