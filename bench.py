@@ -46,6 +46,39 @@ def algorithmic_flops(B, H, N, d, causal):
     return (2 if causal else 4) * B * H * N * N * d
 
 
+def rank_seed(rank):
+    """Each rank runs its own independent prefill: distinct seeded inputs."""
+    import workload
+    return workload.CONFIG_SEED_BASE + 3 + 1000 * rank
+
+
+def reduce_max(x, world, device):
+    """Max over ranks (the slowest rank's time defines the job's time)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(values, world, device):
+    """Element-wise integer sum over ranks (collapse counts)."""
+    if world == 1:
+        return [int(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([int(v) for v in values], dtype=torch.int64, device=device)
+    dist.all_reduce(t)
+    return [int(v) for v in t.tolist()]
+
+
+def job_tflops(flops_per_rank, world, max_ms_per_step):
+    """Whole-job throughput: all ranks' algorithmic work / the slowest rank's time."""
+    return world * flops_per_rank / (max_ms_per_step * 1e-3) / 1e12
+
+
 def peak_tflops():
     """FP8 dense peak: the measured BF16 GEMM burst peak x 2 (nominal fp8/bf16
     ratio), else the machine's fallback figure."""
@@ -136,7 +169,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     fa.load_library()
     import workload
-    W, (q, k, v) = make_inputs(workload.CONFIG_SEED_BASE + 3 + 1000 * rank, dev)
+    W, (q, k, v) = make_inputs(rank_seed(rank), dev)
     B, H, Hkv, N, d = CFG["B"], CFG["H"], CFG["H_kv"], CFG["N"], CFG["d"]
     scale = 1.0 / math.sqrt(d)
     O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
@@ -164,12 +197,7 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return reduce_max(e0.elapsed_time(e1), world, dev)
 
     for _ in range(args.warmup):
         step(True)
@@ -183,7 +211,7 @@ def run_ours(args, rank, world, local_rank):
 
     flops = algorithmic_flops(B, H, N, d, True)
     step_ms = ms_on / args.steps
-    value = world * flops / (step_ms * 1e-3) / 1e12
+    value = job_tflops(flops, world, step_ms)
     kernel_tflops = flops / (step_ms * 1e-3) / 1e12
     peak, peak_src = peak_tflops()
 
@@ -192,8 +220,8 @@ def run_ours(args, rank, world, local_rank):
             return None
         return {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
-                "mode": "kernel only", "value_counter_off":
-                round(world * flops / (ms_off / args.steps * 1e-3) / 1e12, 2)}
+                "mode": "kernel only",
+                "value_counter_off": round(job_tflops(flops, world, ms_off / args.steps), 2)}
 
     # end to end through the public API: pinned host E4M3 inputs -> device ->
     # kernel -> BF16 output back to pinned host memory, every step
@@ -208,14 +236,11 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e2e_steps = max(2, args.steps // 2)
     ms_e2e = timed(e2e_step, e2e_steps)
-    e2e_value = world * flops / (ms_e2e / e2e_steps * 1e-3) / 1e12
+    e2e_value = job_tflops(flops, world, ms_e2e / e2e_steps)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size() + 16
 
-    if world > 1:
-        ct = torch.tensor([collapse_total, collapse_sink], dtype=torch.int64, device=dev)
-        dist.all_reduce(ct)
-        collapse_total, collapse_sink = (int(x) for x in ct.tolist())
+    collapse_total, collapse_sink = reduce_sum([collapse_total, collapse_sink], world, dev)
 
     if rank != 0:
         return None
@@ -229,7 +254,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": WORKLOAD, **CFG, "per_rank": "independent prefill per GPU",
                    "l2": "inputs 201 MB > 126 MB L2, no flush"},
-        "value_counter_off": round(world * flops / (ms_off / args.steps * 1e-3) / 1e12, 2),
+        "value_counter_off": round(job_tflops(flops, world, ms_off / args.steps), 2),
         "pct_of_fp8_peak": {"measured": round(kernel_tflops / peak, 4),
                             "nominal_4500": round(kernel_tflops / 4500.0, 4)},
         "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2),

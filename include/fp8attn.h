@@ -102,6 +102,11 @@ typedef struct {
                                             wait expires writes a nonzero code here and
                                             leaves O incomplete */
   unsigned long long timeout_ns;         /* bound of each wait; 0 = 2 s */
+  int debug_skip_kv_step;                /* testing only, normally 0.  k > 0: the producer
+                                            never issues the K tile of the k-th KV step
+                                            (1-based), so the MMA warp's bounded wait runs
+                                            out, status_word records it and the launch ends
+                                            with O incomplete */
 } fp8attn_params;
 
 int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream);

@@ -34,7 +34,7 @@ class Params(ctypes.Structure):
                 ("o_dtype", ctypes.c_int), ("block_n", ctypes.c_int),
                 ("collapse_ctr", ctypes.c_void_p), ("collapse_sink_ctr", ctypes.c_void_p),
                 ("collapse_rows", ctypes.c_void_p), ("status_word", ctypes.c_void_p),
-                ("timeout_ns", ctypes.c_ulonglong)]
+                ("timeout_ns", ctypes.c_ulonglong), ("debug_skip_kv_step", ctypes.c_int)]
 
 
 # exported symbol -> (argtypes, restype); every symbol of include/fp8attn.h
@@ -120,7 +120,7 @@ def fp8_attn_fwd(Q, K, V, O, B, H, N, d, causal, scale, S, kv_order, n_sink, col
 def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S=256.0,
                     kv_order=KV_REVERSE, n_sink=0, o_dtype=O_BF16, block_n=0,
                     collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None,
-                    status_word=None, timeout_ns=0, stream=None):
+                    status_word=None, timeout_ns=0, debug_skip_kv_step=0, stream=None):
     """Full-parameter entry point (all tensors on the device)."""
     p = Params(Q=Q.data_ptr(), K=K.data_ptr(), V=V.data_ptr(), O=O.data_ptr(),
                B=B, H=H, H_kv=H_kv, N=N, d=d, causal=int(causal),
@@ -131,5 +131,5 @@ def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S
                collapse_sink_ctr=None if collapse_sink_ctr is None else collapse_sink_ctr.data_ptr(),
                collapse_rows=None if collapse_rows is None else collapse_rows.data_ptr(),
                status_word=None if status_word is None else status_word.data_ptr(),
-               timeout_ns=int(timeout_ns))
+               timeout_ns=int(timeout_ns), debug_skip_kv_step=int(debug_skip_kv_step))
     _check(load_library().fp8_attn_fwd_ex(ctypes.byref(p), _stream(stream)), "fp8_attn_fwd_ex")

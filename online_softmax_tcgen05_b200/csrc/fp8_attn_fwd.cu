@@ -50,7 +50,7 @@ constexpr float LOG2E = 1.4426950408889634f;
 // (exp2_poly.cuh) and the rest on MUFU ex2: the two units then share the
 // exponentials of the softmax.
 #ifndef FP8ATTN_POLY_OF_8
-#define FP8ATTN_POLY_OF_8 2
+#define FP8ATTN_POLY_OF_8 0
 #endif
 constexpr int POLY_OF_8 = FP8ATTN_POLY_OF_8;
 
@@ -79,6 +79,7 @@ struct KParams {
   unsigned int* rows;
   unsigned int* status;
   unsigned long long timeout_ns;
+  int debug_skip_kv_step;   // testing hook: 1-based KV step whose K load is never issued
 };
 
 template <int D, int BN>
@@ -181,6 +182,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int st = t % NSTAGE, n = t / NSTAGE;
         if (t >= NSTAGE && !mbar_wait(bar_k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
           return false;
+        if (t + 1 == p.debug_skip_kv_step) return true;   // testing: leave this K tile out
         mbar_arrive_expect_tx(bar_k_full(st), BN * D);
         tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
                     bkv);
@@ -198,8 +200,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     bkv);
         v_issued = t + 1;
       }
-      if (*abort_flag) {
-        // drain: the last load issued into each stage must land before exit
+      {
+        // drain: the last load issued into each stage must land before the CTA
+        // exits (immediate when the consumers took them all; needed after an abort)
         const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8),
                             p.timeout_ns};
         for (int t = k_issued - 1; t >= 0 && t >= k_issued - NSTAGE; --t)
@@ -304,17 +307,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int j = 0; j < BN; ++j)
           if (j0 + j > lim) s[j] = -INFINITY;
       }
-      // row max: 16 independent chains, then a tree
+      // row max: 16 independent chains of three-input max, then a tree
       float mx16[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) mx16[i] = s[i];
 #pragma unroll
-      for (int j = 16; j < BN; ++j) mx16[j & 15] = fmaxf(mx16[j & 15], s[j]);
+      for (int j = 16; j + 16 < BN; j += 32)
 #pragma unroll
-      for (int w = 8; w >= 1; w >>= 1)
+        for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
+      if constexpr ((BN - 16) % 32 != 0) {
 #pragma unroll
-        for (int i = 0; i < w; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + w]);
-      const float m_new = fmaxf(m_run, mx16[0] * c);
+        for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
+      }
+      float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
+                       fmax3(mx16[6], mx16[7], mx16[8]));
+      mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
+      mx = fmaxf(mx, mx16[15]);
+      const float m_new = fmaxf(m_run, mx * c);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
       // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
@@ -623,6 +632,9 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   if (p->n_sink < 0 || p->n_sink > p->N) return fail(FP8ATTN_EINVAL, "n_sink must be in [0, N]");
   if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
     return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
+  if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
+  if (p->debug_skip_kv_step > 0 && !p->status_word)
+    return fail(FP8ATTN_EINVAL, "debug_skip_kv_step needs a status_word to report the timeout");
   if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
     return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
   if ((long long)p->B * p->H > 65535LL * 65535LL) return fail(FP8ATTN_EINVAL, "B*H too large");
@@ -661,6 +673,7 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.rows = p->collapse_rows;
   kp.status = p->status_word;
   kp.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
+  kp.debug_skip_kv_step = p->debug_skip_kv_step;
   if (kp.B * kp.H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
 
   const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;

@@ -54,7 +54,7 @@ def base_params(**kw):
     p = dict(Q=FAKE, K=FAKE, V=FAKE, O=FAKE, B=1, H=2, H_kv=1, N=256, d=128, causal=0,
              scale=0.088, S=256.0, kv_order=1, n_sink=4, o_dtype=0, block_n=0,
              collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None, status_word=None,
-             timeout_ns=0)
+             timeout_ns=0, debug_skip_kv_step=0)
     p.update(kw)
     return Params(**p)
 
@@ -68,6 +68,7 @@ def base_params(**kw):
     (dict(n_sink=257), EINVAL), (dict(o_dtype=5), EINVAL), (dict(Q=None), EINVAL),
     (dict(O=FAKE + 8), EINVAL), (dict(K=FAKE + 1), EINVAL),
     (dict(collapse_rows=FAKE), EINVAL), (dict(collapse_ctr=FAKE + 4), EINVAL),
+    (dict(debug_skip_kv_step=-1), EINVAL), (dict(debug_skip_kv_step=2), EINVAL),
 ])
 def test_invalid_arguments_rejected_before_launch(lib, kw, status):
     p = base_params(**kw)

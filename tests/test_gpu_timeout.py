@@ -1,0 +1,39 @@
+"""Failure detection on the GPU without a fault: every mbarrier wait of the
+attention kernel is bounded in time.  The test-only hook debug_skip_kv_step
+leaves one K tile unloaded, so the MMA warp's wait for it can only run out;
+the kernel must then record where in the status word, free its TMEM and
+return, leaving the context usable for the next launch."""
+import math
+
+import numpy as np
+import pytest
+
+from helpers import assert_o_close, gpu_inputs, oracle, workload
+
+pytestmark = pytest.mark.gpu
+
+
+def test_expired_wait_reports_status_and_context_survives():
+    import torch
+    from online_softmax_tcgen05_b200 import O_F32, device_status_string, fp8_attn_fwd_ex
+    B, H, N, d = 1, 1, 512, 128
+    W = workload.make_sink_workload(B, H, H, N, d, 4, 8.0, seed=9)
+    ins = gpu_inputs(W)
+    (q, Q8), (k, K8), (v, V8) = ins
+    O = torch.zeros((B, H, N, d), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=H, N=N, d=d, S=256.0, kv_order=1, n_sink=4,
+                    o_dtype=O_F32, status_word=status, timeout_ns=50_000_000,
+                    debug_skip_kv_step=2)
+    torch.cuda.synchronize()
+    word = int(status.item())
+    assert word == 0x103, hex(word)                 # MMA warp gave up waiting for a K tile
+    assert "K tile" in device_status_string(word)
+    # the same context runs a normal launch correctly afterwards
+    status.zero_()
+    fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=H, N=N, d=d, S=256.0, kv_order=1, n_sink=4,
+                    o_dtype=O_F32, status_word=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    Oe, _, _ = oracle.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, 1 / math.sqrt(d), 256.0, 1, 128, 4)
+    assert_o_close(O.cpu().numpy().reshape(-1, d), Oe, "after timeout")
