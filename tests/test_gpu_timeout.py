@@ -27,8 +27,10 @@ def test_expired_wait_reports_status_and_context_survives():
                     debug_skip_kv_step=2)
     torch.cuda.synchronize()
     word = int(status.item())
-    assert word == 0x103, hex(word)                 # MMA warp gave up waiting for a K tile
-    assert "K tile" in device_status_string(word)
+    # the first wait to run out is either the MMA warp's (the K tile never lands)
+    # or the producer's (the stage that tile's QK^T would free never frees)
+    assert word in (0x101, 0x103), hex(word)
+    assert device_status_string(word).startswith("timeout")
     # the same context runs a normal launch correctly afterwards
     status.zero_()
     fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=H, N=N, d=d, S=256.0, kv_order=1, n_sink=4,
