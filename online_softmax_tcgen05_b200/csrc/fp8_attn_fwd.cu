@@ -42,10 +42,11 @@
 
 namespace fp8attn {
 
-constexpr int BM = 128;          // query rows per tile (= MMA M, = TMEM lanes)
-constexpr int NTILE = 2;         // query tiles per CTA, sharing one K/V stream
-constexpr int NSTAGE = 3;        // K/V ring depth
-constexpr int NTHREADS = 512;    // softmax WG x2, correction WG, producer / MMA WG
+constexpr int BM = 128;         // query rows per CTA (= MMA M, = TMEM lanes)
+constexpr int NSTAGE = 2;       // K/V ring depth
+constexpr int NSPLIT = 2;       // softmax threads per query row (each owns block_n / 2 keys)
+constexpr int NSOFTMAX = 4 * NSPLIT;            // softmax warps
+constexpr int NTHREADS = 32 * (NSOFTMAX + 2);   // + TMA warp + MMA warp
 constexpr float LOG2E = 1.4426950408889634f;
 // Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
 // (exp2_poly.cuh) and the rest on MUFU ex2: the two units then share the
@@ -66,14 +67,12 @@ enum : uint32_t {
   WAIT_SM_S_FULL = 7,
   WAIT_SM_O_DONE = 8,
   WAIT_EPI_O_DONE = 9,
-  WAIT_CORR_P = 10,
-  WAIT_CORR_O_DONE = 11,
 };
 
 struct KParams {
   int B, H, Hkv, N, group;
   int causal, kv_order, n_sink;
-  int num_q_blocks;   // CTAs along the sequence: ceil(N / (NTILE * BM))
+  int num_q_tiles;
   float scale_log2;   // scale * log2(e)
   float S;
   void* O;
@@ -85,41 +84,25 @@ struct KParams {
   int debug_skip_kv_step;   // testing hook: 1-based KV step whose K load is never issued
 };
 
-// Shared-memory map of one CTA (offsets from a 1024-aligned base).
 template <int D, int BN>
 struct Smem {
-  static constexpr int Q = 0;                               // [tile] BM x D
-  static constexpr int K = Q + NTILE * BM * D;              // [stage] BN x D
-  static constexpr int V = K + NSTAGE * BN * D;             // [stage] BN x D
-  static constexpr int P = V + NSTAGE * BN * D;             // [tile][buffer] BM x BN
-  static constexpr int ALPHA = P + NTILE * 2 * BM * BN;     // float [tile][buffer][BM]
-  static constexpr int LSUM = ALPHA + NTILE * 2 * BM * 4;   // float [tile][BM]
-  static constexpr int BAR = LSUM + NTILE * BM * 4;
-  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[T], s_free[T],
-  // p_full[T][2], o_ready[T], o_done[T][2], drain
-  static constexpr int NBAR = 1 + 4 * NSTAGE + NTILE * 7 + 1;
-  static constexpr int MISC = BAR + 8 * NBAR;               // tmem slot, abort flag, drain flag
+  static constexpr int Q = 0;
+  static constexpr int K = Q + BM * D;
+  static constexpr int V = K + NSTAGE * BN * D;
+  static constexpr int P = V + NSTAGE * BN * D;
+  static constexpr int XMAX = P + BM * BN;                  // float [2 buffers][NSPLIT][BM]
+  static constexpr int XFIN = XMAX + 2 * NSPLIT * BM * 4;   // float l, uint count [NSPLIT][BM]
+  static constexpr int BAR = XFIN + 2 * NSPLIT * BM * 4;
+  // barriers: q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full, s_free, p_full,
+  // o_done, drain, xch[4 quarters][2 buffers], fin[4 quarters]
+  static constexpr int NBAR = 1 + 4 * NSTAGE + 5 + 4 * 2 + 4;
+  static constexpr int MISC = BAR + 8 * NBAR;   // tmem base slot, abort flag, drain flag
   static constexpr int BYTES = MISC + 16;
-  static constexpr int ALLOC = BYTES + 1024;
-  static constexpr uint32_t TMEM_COLS = 512;                // S_A, S_B, O_A, O_B
-  static_assert(NTILE * (BN + D) <= (int)TMEM_COLS, "TMEM budget");
-  static_assert(ALLOC <= 227 * 1024, "shared memory budget");
-};
-
-struct Bars {
-  uint32_t base;
-  __device__ uint32_t q_full() const { return base; }
-  __device__ uint32_t k_full(int s) const { return base + 8u * (1 + s); }
-  __device__ uint32_t k_empty(int s) const { return base + 8u * (1 + NSTAGE + s); }
-  __device__ uint32_t v_full(int s) const { return base + 8u * (1 + 2 * NSTAGE + s); }
-  __device__ uint32_t v_empty(int s) const { return base + 8u * (1 + 3 * NSTAGE + s); }
-  __device__ uint32_t tile0() const { return base + 8u * (1 + 4 * NSTAGE); }
-  __device__ uint32_t s_full(int x) const { return tile0() + 8u * (7 * x + 0); }
-  __device__ uint32_t s_free(int x) const { return tile0() + 8u * (7 * x + 1); }
-  __device__ uint32_t p_full(int x, int b) const { return tile0() + 8u * (7 * x + 2 + b); }
-  __device__ uint32_t o_ready(int x) const { return tile0() + 8u * (7 * x + 4); }
-  __device__ uint32_t o_done(int x, int b) const { return tile0() + 8u * (7 * x + 5 + b); }
-  __device__ uint32_t drain() const { return tile0() + 8u * (7 * NTILE); }
+  // slack to align the base to 1024, and at least 80 KB so that no more than two
+  // CTAs share an SM: two 256-column TMEM allocations fill the SM's 512 columns
+  static constexpr int ALLOC = (BYTES + 1024 > 80 * 1024) ? BYTES + 1024 : 80 * 1024;
+  static constexpr uint32_t TMEM_COLS = 256;    // S: BN columns, O: D columns
+  static_assert(BN + D <= (int)TMEM_COLS, "TMEM budget");
 };
 
 __device__ __forceinline__ int kv_block_at(int t, int T, int order) {
@@ -131,109 +114,61 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl, where));
 }
 
-// One KV block of the online softmax for one query row (Problem statement of
-// the P-cast paper): row max over the block, rescale factor alpha, p = 2^(s*c - m),
-// FP32 row sum before the cast, S*p cast to E4M3 (packed four keys per word),
-// and the collapse count of the block.  s[] holds the raw QK^T dot products.
-template <int BN, bool COUNT>
-__device__ __forceinline__ void softmax_block(float (&s)[BN], int j0, int lim, bool need_mask,
-                                              int n_sink, float c, float S, float& m_run,
-                                              float& l, float& alpha, uint32_t (&pw)[BN / 4],
-                                              uint32_t& cnt, uint32_t& cnt_sink) {
-  if (need_mask) {
+// The NSPLIT softmax warps that share one TMEM lane quarter (the parts of the
+// same 32 rows) meet on an mbarrier of count NSPLIT: each warp publishes its
+// values in shared memory, arrives once, and waits (bounded, abort-aware) for
+// the others.
+__device__ __forceinline__ bool pair_exchange(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
+                                              int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  return warp_wait(bar, parity, ctl, 0x20);
+}
+
+// Largest of n values, 8 independent chains then a tree.
+template <int N>
+__device__ __forceinline__ float row_max(const float (&s)[N]) {
+  float m8[8];
 #pragma unroll
-    for (int j = 0; j < BN; ++j)
-      if (j0 + j > lim) s[j] = -INFINITY;
-  }
-  // row max: 16 independent chains of three-input max, then a tree
-  float mx16[16];
+  for (int i = 0; i < 8; ++i) m8[i] = s[i];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) mx16[i] = s[i];
-#pragma unroll
-  for (int j = 16; j + 16 < BN; j += 32)
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
-  if constexpr ((BN - 16) % 32 != 0) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
-  }
-  float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
-                   fmax3(mx16[6], mx16[7], mx16[8]));
-  mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
-  mx = fmaxf(mx, mx16[15]);
-  const float m_new = fmaxf(m_run, mx * c);
-  const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-  alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-  m_run = m_new;
-  // p = 2^(s*c - m): packed FFMA2 for the argument, then MUFU ex2 (or the
-  // FMA-pipe polynomial for POLY_OF_8 of every 8 pairs), split packed row sums
-  const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
-  float2 acc8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int q = 0; q < BN / 2; ++q) {
-    const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
-    if ((q & 7) < POLY_OF_8) {
-      const float2 e = exp2_poly2(y);
-      s[2 * q] = e.x;
-      s[2 * q + 1] = e.y;
-    } else {
-      s[2 * q] = ex2_approx(y.x);
-      s[2 * q + 1] = ex2_approx(y.y);
-    }
-    acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
-  }
+  for (int j = 8; j < N; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
 #pragma unroll
   for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
-    for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
-  l = alpha * l + (acc8[0].x + acc8[0].y);
-  // S * p (packed FMUL2), then the E4M3 cast, four keys per word
-  const float2 S2 = make_float2(S, S);
-#pragma unroll
-  for (int q = 0; q < BN / 4; ++q) {
-    const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
-    const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
-    pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
-  }
-  if constexpr (COUNT) {
-    // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
-    // negative, so byte 0 <=> the cast flushed S*p to zero.  Zero bytes are found
-    // four at a time; blocks that hold a sink or a masked key restrict the count
-    // to the lanes with n_sink <= j <= last visible key.
-    uint32_t zacc = 0;
-    if (j0 >= n_sink && !need_mask) {
-#pragma unroll
-      for (int q = 0; q < BN / 4; ++q) {
-        const uint32_t w = pw[q];
-        zacc += ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu) >> 7;
-      }
-    } else {
-      const int lo = max(n_sink - j0, 0), hi = min(lim - j0, BN - 1);   // block-local
-#pragma unroll
-      for (int q = 0; q < BN / 4; ++q) {
-        const uint32_t w = pw[q];
-        const uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
-        const int a = lo - 4 * q, bq = hi - 4 * q;   // lanes a..bq of this word are valid
-        const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
-        const uint32_t mhi =
-            bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
-        zacc += (y & mlo & mhi) >> 7;
-      }
-    }
-    const uint32_t cblk = (zacc * 0x01010101u) >> 24;   // byte lanes hold <= BN/4 each
-    cnt += cblk;
-    if (j0 < n_sink) cnt_sink += cblk;
-  }
+    for (int i = 0; i < w; ++i) m8[i] = fmaxf(m8[i], m8[i + w]);
+  return m8[0];
 }
 
-// O (D TMEM columns of this warp's 32 rows) *= alpha, 32 columns per round trip.
-template <int D>
+// Number of zero bytes among the valid lanes of HC/4 packed E4M3 words
+// (collapse count of one part of a row).  Valid keys: block-local index in
+// [lo, hi]; all_valid skips the lane masks.  Four independent accumulators.
+template <int HC>
+__device__ __forceinline__ uint32_t zero_bytes(const uint32_t (&pw)[HC / 4], int k0, int lo, int hi,
+                                               bool all_valid) {
+  uint32_t z[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int q = 0; q < HC / 4; ++q) {
+    const uint32_t w = pw[q];
+    uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
+    if (!all_valid) {
+      const int a = lo - (k0 + 4 * q), bq = hi - (k0 + 4 * q);   // valid lanes a..bq of the word
+      const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
+      const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
+      y &= mlo & mhi;
+    }
+    z[q & 3] += y >> 7;   // one count per byte lane
+  }
+  const uint32_t zs = (z[0] + z[1]) + (z[2] + z[3]);   // byte lanes hold <= HC/4 each
+  return (zs * 0x01010101u) >> 24;
+}
+
+// O (NC TMEM columns of this warp's 32 rows) *= alpha, 32 columns per round trip.
+template <int NC>
 __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
   const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-  for (int cc = 0; cc < D / 32; ++cc) {
+  for (int cc = 0; cc < NC / 32; ++cc) {
     uint32_t o[32];
     tmem_ld32(tO + 32 * cc, o);
     tmem_wait_ld();
@@ -249,13 +184,13 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
   tmem_wait_st();
 }
 
-// Epilogue of one row: O / (S l) from TMEM to global memory (BF16 RNE or FP32),
-// 32 columns at a time, divided in place.
-template <int D, bool OUT_BF16>
+// Epilogue of one row part: NC columns of O / (S l) from TMEM to global memory
+// (BF16 RNE or FP32), 32 columns at a time, divided in place.
+template <int NC, bool OUT_BF16>
 __device__ __forceinline__ void store_row(uint32_t tO, float denom, bool live, void* O,
                                           size_t obase) {
-#pragma unroll 1
-  for (int cc = 0; cc < D / 32; ++cc) {
+#pragma unroll
+  for (int cc = 0; cc < NC / 32; ++cc) {
     uint32_t o[32];
     tmem_ld32(tO + 32 * cc, o);
     tmem_wait_ld();
@@ -277,74 +212,92 @@ __device__ __forceinline__ void store_row(uint32_t tO, float denom, bool live, v
       } else {
         uint4* out = reinterpret_cast<uint4*>(static_cast<float*>(O) + obase + 32 * cc);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) out[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        for (int k = 0; k < 8; ++k)
+          out[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
       }
     }
   }
 }
 
-// One CTA = two 128-row query tiles (A: rows q0.., B: rows q0+128..) of one
-// (batch, head), both streaming the same K/V blocks in the visiting order.
-//   warps 0-3, 4-7  softmax of tile A, tile B (one thread per row)
-//   warps 8-11      correction: O rescale by alpha between P~V steps, epilogue
-//   warp 12         TMA producer (Q tiles once; K, V ring; K one step ahead)
-//   warp 13         MMA issuer and TMEM owner; warps 14, 15 idle
-// TMEM: S_A [0,BN), S_B [BN,2BN), O_A [2BN,2BN+D), O_B [2BN+D,2BN+2D).
+// One CTA = one 128-row query tile of one (batch, head); two CTAs share an SM.
+//   warps 0-7  softmax: warp w holds rows 32(w%4)..+31 (its TMEM lane quarter)
+//              and keys [w/4 * BN/2, (w/4 + 1) * BN/2) of each KV block, and
+//              columns [w/4 * D/2, (w/4 + 1) * D/2) of O; the two warps of a
+//              quarter exchange their partial row maxima each block
+//   warp 8     TMA producer: Q tile once, K and V of each KV block in visiting
+//              order into a 2-stage ring, K one step ahead of V
+//   warp 9     MMA issuer and TMEM owner: S = Q K^T, O += P~ V
+// TMEM: S [0, BN), O [BN, BN + D).
 template <int D, int BN, bool OUT_BF16, bool COUNT>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(NTHREADS, 2)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p) {
   using L = Smem<D, BN>;
+  constexpr int HC = BN / NSPLIT;   // keys per softmax thread
+  constexpr int OC = D / NSPLIT;    // O columns per softmax thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::Q, sK = sbase + L::K, sV = sbase + L::V, sP = sbase + L::P;
-  float* alpha_sm = reinterpret_cast<float*>(smem + L::ALPHA);
-  float* lsum_sm = reinterpret_cast<float*>(smem + L::LSUM);
-  const Bars bars{sbase + L::BAR};
+  float* xmax = reinterpret_cast<float*>(smem + L::XMAX);
+  float* xl = reinterpret_cast<float*>(smem + L::XFIN);
+  uint32_t* xcnt = reinterpret_cast<uint32_t*>(smem + L::XFIN + NSPLIT * BM * 4);
+  const uint32_t bar0 = sbase + L::BAR;
+  const uint32_t bar_q_full = bar0;
+  auto bar_k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_v_full = [&](int s) { return bar0 + 8u * (1 + NSTAGE + s); };
+  auto bar_k_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NSTAGE + s); };
+  auto bar_v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * NSTAGE + s); };
+  const uint32_t bar_s_full = bar0 + 8u * (1 + 4 * NSTAGE);
+  const uint32_t bar_s_free = bar_s_full + 8;
+  const uint32_t bar_p_full = bar_s_full + 16;
+  const uint32_t bar_o_done = bar_s_full + 24;
+  const uint32_t bar_drain = bar_s_full + 32;
+  auto bar_xch = [&](int quarter, int buf) { return bar_s_full + 40 + 8u * (2 * quarter + buf); };
+  auto bar_fin = [&](int quarter) { return bar_s_full + 40 + 64 + 8u * quarter; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 4);
   volatile uint32_t* never_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = p.causal ? (p.num_q_blocks - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int tile = p.causal ? (p.num_q_tiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
   const int bh = blockIdx.y;
   const int h = bh % p.H, b = bh / p.H;
   const int bkv = b * p.Hkv + h / p.group;
-  const int q0 = qb * NTILE * BM;
-  const int last_row = min(q0 + NTILE * BM - 1, p.N - 1);
+  const int q0 = tile * BM;
+  const int last_row = min(q0 + BM - 1, p.N - 1);
   const int T = p.causal ? (last_row / BN + 1) : ((p.N + BN - 1) / BN);
   const WaitCtl ctl{abort_flag, p.timeout_ns};
   const WaitCtl drain{never_flag, p.timeout_ns};
 
   if (threadIdx.x == 0) {
-    mbar_init(bars.q_full(), 1);
+    mbar_init(bar_q_full, 1);
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(bars.k_full(s), 1);
-      mbar_init(bars.k_empty(s), 1);
-      mbar_init(bars.v_full(s), 1);
-      mbar_init(bars.v_empty(s), 1);
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+      mbar_init(bar_v_empty(s), 1);
     }
-    for (int x = 0; x < NTILE; ++x) {
-      mbar_init(bars.s_full(x), 1);
-      mbar_init(bars.s_free(x), 4);
-      mbar_init(bars.p_full(x, 0), 4);
-      mbar_init(bars.p_full(x, 1), 4);
-      mbar_init(bars.o_ready(x), 4);
-      mbar_init(bars.o_done(x, 0), 1);
-      mbar_init(bars.o_done(x, 1), 1);
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_s_free, NSOFTMAX);
+    mbar_init(bar_p_full, NSOFTMAX);
+    mbar_init(bar_o_done, 1);
+    mbar_init(bar_drain, 1);
+    for (int qd = 0; qd < 4; ++qd) {
+      mbar_init(bar_xch(qd, 0), NSPLIT);
+      mbar_init(bar_xch(qd, 1), NSPLIT);
+      mbar_init(bar_fin(qd), NSPLIT);
     }
-    mbar_init(bars.drain(), 1);
     *abort_flag = 0;
     *never_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 13) {
+  if (warp == NSOFTMAX + 1) {
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 12 && lane == 0) {
+  if (warp == NSOFTMAX && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -354,24 +307,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp >= 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
-    if (warp == 12 && lane == 0) {
-      // ---------------------------------------------------------- producer --
-      mbar_arrive_expect_tx(bars.q_full(), NTILE * BM * D);
-      for (int x = 0; x < NTILE; ++x)
-        tma_load_3d(sQ + x * BM * D, &tmQ, bars.q_full(), 0, q0 + x * BM, bh);
-      // K runs one KV step ahead of V: K(t+1) needs only QK^T(t+1-NSTAGE) to have
-      // released its stage, V(t) needs P~V(t-NSTAGE).
+  if (warp == NSOFTMAX) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q_full, BM * D);
+      tma_load_3d(sQ, &tmQ, bar_q_full, 0, q0, bh);
+      // K runs one KV step ahead of V: K(t+1) needs only QK^T(t-1) to have
+      // released its stage, V(t) needs P~V(t-2).
       int k_issued = 0, v_issued = 0;
       auto load_k = [&](int t) -> bool {
         const int st = t % NSTAGE, n = t / NSTAGE;
-        if (t >= NSTAGE && !mbar_wait(bars.k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+        if (t >= NSTAGE && !mbar_wait(bar_k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
           return false;
         if (t + 1 == p.debug_skip_kv_step) return true;   // testing: leave this K tile out
-        mbar_arrive_expect_tx(bars.k_full(st), BN * D);
-        tma_load_3d(sK + st * BN * D, &tmK, bars.k_full(st), 0,
-                    kv_block_at(t, T, p.kv_order) * BN, bkv);
+        mbar_arrive_expect_tx(bar_k_full(st), BN * D);
+        tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
+                    bkv);
         k_issued = t + 1;
         return true;
       };
@@ -379,177 +330,208 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int t = 0; ok && t < T; ++t) {
         if (t + 1 < T && !load_k(t + 1)) break;
         const int st = t % NSTAGE, n = t / NSTAGE;
-        if (t >= NSTAGE && !mbar_wait(bars.v_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+        if (t >= NSTAGE && !mbar_wait(bar_v_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
           break;
-        mbar_arrive_expect_tx(bars.v_full(st), BN * D);
-        tma_load_3d(sV + st * BN * D, &tmV, bars.v_full(st), 0,
-                    kv_block_at(t, T, p.kv_order) * BN, bkv);
+        mbar_arrive_expect_tx(bar_v_full(st), BN * D);
+        tma_load_3d(sV + st * BN * D, &tmV, bar_v_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
+                    bkv);
         v_issued = t + 1;
       }
       // drain: the last load issued into each stage must land before the CTA
       // exits (immediate when the consumers took them all; needed after an abort)
       for (int t = k_issued - 1; t >= 0 && t >= k_issued - NSTAGE; --t)
-        mbar_wait(bars.k_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
+        mbar_wait(bar_k_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
       for (int t = v_issued - 1; t >= 0 && t >= v_issued - NSTAGE; --t)
-        mbar_wait(bars.v_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
-      mbar_wait(bars.q_full(), 0, drain, 0);
-    } else if (warp == 13) {
-      // --------------------------------------------------------------- MMA --
-      constexpr uint32_t SWZ_QK = (D == 128) ? SWZ_128B : SWZ_64B;
-      constexpr uint32_t SWZ_P = (BN == 128) ? SWZ_128B : SWZ_64B;
-      constexpr uint32_t IDESC_QK = idesc_e4m3_f32(BM, BN, 0, 0);
-      constexpr uint32_t IDESC_PV = idesc_e4m3_f32(BM, D, 0, 1);
-      bool ok = mbar_wait(bars.q_full(), 0, ctl, WAIT_MMA_Q);
-      for (int t = 0; ok && t <= T; ++t) {
-        if (t < T) {
-          const int st = t % NSTAGE;
-          ok = mbar_wait(bars.k_full(st), (t / NSTAGE) & 1, ctl, WAIT_MMA_K);
-          for (int x = 0; ok && x < NTILE; ++x) {
-            if (t > 0) ok = mbar_wait(bars.s_free(x), (t - 1) & 1, ctl, WAIT_MMA_S_FREE);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
+        mbar_wait(bar_v_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
+      mbar_wait(bar_q_full, 0, drain, 0);
+    }
+  } else if (warp == NSOFTMAX + 1) {
+    // ----------------------------------------------------------------- MMA --
+    constexpr uint32_t SWZ_QK = (D == 128) ? SWZ_128B : SWZ_64B;
+    constexpr uint32_t SWZ_P = (BN == 128) ? SWZ_128B : SWZ_64B;
+    constexpr uint32_t IDESC_QK = idesc_e4m3_f32(BM, BN, 0, 0);
+    constexpr uint32_t IDESC_PV = idesc_e4m3_f32(BM, D, 0, 1);
+    const uint32_t tS = tmem_base, tO = tmem_base + BN;
+    bool ok = mbar_wait(bar_q_full, 0, ctl, WAIT_MMA_Q);
+    auto issue_qk = [&](int st) {
+      tc_fence_after();
+      if (lane == 0) {
 #pragma unroll
-              for (int kk = 0; kk < D / 32; ++kk) {
-                const uint64_t a = smem_desc(sQ + x * BM * D + 32 * kk, 16, 8 * D, SWZ_QK);
-                const uint64_t bd = smem_desc(sK + st * BN * D + 32 * kk, 16, 8 * D, SWZ_QK);
-                mma_e4m3_ss(tmem_base + x * BN, a, bd, IDESC_QK, kk > 0);
-              }
-              mma_commit(bars.s_full(x));
-            }
-            __syncwarp();
-          }
-          if (!ok) break;
-          if (lane == 0) mma_commit(bars.k_empty(st));
-          __syncwarp();
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t a = smem_desc(sQ + 32 * kk, 16, 8 * D, SWZ_QK);
+          const uint64_t bdesc = smem_desc(sK + st * BN * D + 32 * kk, 16, 8 * D, SWZ_QK);
+          mma_e4m3_ss(tS, a, bdesc, IDESC_QK, kk > 0);
         }
-        if (t > 0) {
-          const int u = t - 1, st = u % NSTAGE;
-          ok = mbar_wait(bars.v_full(st), (u / NSTAGE) & 1, ctl, WAIT_MMA_V);
-          for (int x = 0; ok && x < NTILE; ++x) {
-            ok = mbar_wait(bars.o_ready(x), u & 1, ctl, WAIT_MMA_P);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
-              const uint32_t pbuf = sP + (x * 2 + (u & 1)) * BM * BN;
-#pragma unroll
-              for (int kk = 0; kk < BN / 32; ++kk) {
-                const uint64_t a = smem_desc(pbuf + 32 * kk, 16, 8 * BN, SWZ_P);
-                const uint64_t bd =
-                    smem_desc(sV + st * BN * D + kk * 32 * D, BN * D, 8 * D, SWZ_QK);
-                mma_e4m3_ss(tmem_base + NTILE * BN + x * D, a, bd, IDESC_PV,
-                            (u > 0 || kk > 0) ? 1u : 0u);
-              }
-              mma_commit(bars.o_done(x, u & 1));
-            }
-            __syncwarp();
-          }
-          if (!ok) break;
-          if (lane == 0) mma_commit(bars.v_empty(st));
-          __syncwarp();
-        }
+        mma_commit(bar_s_full);
+        mma_commit(bar_k_empty(st));
       }
-      // drain every MMA this warp issued before TMEM is released
-      if (lane == 0) mma_commit(bars.drain());
       __syncwarp();
-      mbar_wait(bars.drain(), 0, drain, 0);
-    }
-  } else if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
-    // ------------------------------------------------------------ correction --
-    const int r = threadIdx.x - 256;                 // row within each tile
-    const uint32_t lane_off = (uint32_t)(32 * (warp - 8)) << 16;
-    bool ok = true;
+    };
+    if (ok) ok = mbar_wait(bar_k_full(0), 0, ctl, WAIT_MMA_K);
+    if (ok) issue_qk(0);
     for (int t = 0; ok && t < T; ++t) {
-      for (int x = 0; x < NTILE; ++x) {
-        ok = warp_wait(bars.p_full(x, t & 1), (t >> 1) & 1, ctl, WAIT_CORR_P);
+      if (t + 1 < T) {
+        const int st1 = (t + 1) % NSTAGE, ph1 = ((t + 1) / NSTAGE) & 1;
+        ok = mbar_wait(bar_k_full(st1), ph1, ctl, WAIT_MMA_K) &&
+             mbar_wait(bar_s_free, t & 1, ctl, WAIT_MMA_S_FREE);
         if (!ok) break;
-        if (t > 0) {
-          ok = warp_wait(bars.o_done(x, (t - 1) & 1), ((t - 1) >> 1) & 1, ctl, WAIT_CORR_O_DONE);
-          if (!ok) break;
-          tc_fence_after();
-          const float alpha = alpha_sm[(x * 2 + (t & 1)) * BM + r];
-          if (__any_sync(0xffffffffu, alpha != 1.f))
-            rescale_o<D>(tmem_base + lane_off + NTILE * BN + x * D, alpha);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars.o_ready(x));
+        issue_qk(st1);
       }
-    }
-    // epilogue: O / (S l) for both tiles
-    for (int x = 0; ok && x < NTILE; ++x) {
-      ok = warp_wait(bars.o_done(x, (T - 1) & 1), ((T - 1) >> 1) & 1, ctl, WAIT_EPI_O_DONE);
+      const int st = t % NSTAGE, ph = (t / NSTAGE) & 1;
+      ok = mbar_wait(bar_v_full(st), ph, ctl, WAIT_MMA_V) &&
+           mbar_wait(bar_p_full, t & 1, ctl, WAIT_MMA_P);
       if (!ok) break;
       tc_fence_after();
-      const int row = q0 + x * BM + r;
-      const bool live = row < p.N;
-      const float denom = p.S * lsum_sm[x * BM + r];
-      store_row<D, OUT_BF16>(tmem_base + lane_off + NTILE * BN + x * D, denom, live, p.O,
-                             ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D);
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 32; ++kk) {
+          const uint64_t a = smem_desc(sP + 32 * kk, 16, 8 * BN, SWZ_P);
+          const uint64_t bdesc = smem_desc(sV + st * BN * D + kk * 32 * D, BN * D, 8 * D, SWZ_QK);
+          mma_e4m3_ss(tO, a, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar_o_done);
+        mma_commit(bar_v_empty(st));
+      }
+      __syncwarp();
     }
+    // drain every MMA this warp issued before TMEM is released
+    if (lane == 0) mma_commit(bar_drain);
+    __syncwarp();
+    mbar_wait(bar_drain, 0, drain, 0);
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 184;\n" ::: "memory");
-    // --------------------------------------------------------------- softmax --
-    const int x = warp >> 2;                        // tile
-    const int r = threadIdx.x - 128 * x;            // row within the tile
-    const int row = q0 + x * BM + r;
-    const uint32_t tS = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + x * BN;
+    // ------------------------------------------------------------- softmax --
+    const int quarter = warp & 3, part = warp >> 2;
+    const int r = 32 * quarter + lane;            // row within the tile
+    const int row = q0 + r;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t tS = tmem_base + lane_off + part * HC;
+    const uint32_t tO = tmem_base + lane_off + BN + part * OC;
     const float c = p.scale_log2;
+    const float S = p.S;
     float m_run = -INFINITY, l = 0.f;
     uint32_t cnt = 0, cnt_sink = 0;
     bool ok = true;
-    // this thread's P~ row in the swizzled tile (128B swizzle for 128-byte rows,
-    // 64B swizzle for 64-byte rows)
-    const uint32_t prow = sP + x * 2 * BM * BN + (r >> 3) * (8 * BN) + (r & 7) * BN;
+    // this thread's part of the P~ row in the swizzled tile (128B swizzle for
+    // 128-byte rows, 64B swizzle for 64-byte rows)
+    const uint32_t prow = sP + (r >> 3) * (8 * BN) + (r & 7) * BN;
     const uint32_t pswz = (BN == 128) ? (uint32_t)(r & 7) : (uint32_t)((r & 7) >> 1);
     const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
-    const int tile_row0 = q0 + x * BM;
+    const int k0 = part * HC;                                  // first key of this part
 
     for (int t = 0; t < T; ++t) {
       const int j0 = kv_block_at(t, T, p.kv_order) * BN;
-      ok = warp_wait(bars.s_full(x), t & 1, ctl, WAIT_SM_S_FULL);
+      ok = warp_wait(bar_s_full, t & 1, ctl, WAIT_SM_S_FULL);
       if (!ok) break;
       tc_fence_after();
-      float s[BN];
+      float s[HC];
 #pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc)
+      for (int cc = 0; cc < HC / 32; ++cc)
         tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * cc]));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.s_free(x));
+      if (lane == 0) mbar_arrive(bar_s_free);
 
-      const bool need_mask = (p.causal && j0 + BN - 1 > tile_row0) || (j0 + BN > p.N);
-      float alpha;
-      uint32_t pw[BN / 4];
-      softmax_block<BN, COUNT>(s, j0, lim, need_mask, p.n_sink, c, p.S, m_run, l, alpha, pw, cnt,
-                               cnt_sink);
-
-      // P~ buffer t&1 is free once P~V(t-2) of this tile is done
-      if (t >= 2) {
-        ok = warp_wait(bars.o_done(x, t & 1), ((t >> 1) - 1) & 1, ctl, WAIT_SM_O_DONE);
-        if (!ok) break;
-      }
-      const uint32_t pb = prow + (t & 1) * BM * BN;
+      const bool need_mask = (p.causal && j0 + BN - 1 > q0) || (j0 + BN > p.N);
+      if (need_mask) {
 #pragma unroll
-      for (int q = 0; q < BN / 16; ++q) {
-        const uint32_t dst = pb + ((q ^ pswz) << 4);
+        for (int j = 0; j < HC; ++j)
+          if (j0 + k0 + j > lim) s[j] = -INFINITY;
+      }
+      // row max: this part's, then the partner's through shared memory
+      float* xm = xmax + (t & 1) * NSPLIT * BM;
+      xm[part * BM + r] = row_max<HC>(s);
+      ok = pair_exchange(bar_xch(quarter, t & 1), (t >> 1) & 1, ctl, lane);
+      if (!ok) break;
+      float mx = xm[r];
+#pragma unroll
+      for (int q = 1; q < NSPLIT; ++q) mx = fmaxf(mx, xm[q * BM + r]);
+      const float m_new = fmaxf(m_run, mx * c);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
+      m_run = m_new;
+      // p = 2^(s*c - m): packed FFMA2 for the argument, then MUFU ex2 (or the
+      // FMA-pipe polynomial for POLY_OF_8 of every 8 pairs), split packed row sums
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+      float2 acc4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc4[i] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < HC / 2; ++q) {
+        const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
+        if ((q & 7) < POLY_OF_8) {
+          const float2 e = exp2_poly2(y);
+          s[2 * q] = e.x;
+          s[2 * q + 1] = e.y;
+        } else {
+          s[2 * q] = ex2_approx(y.x);
+          s[2 * q + 1] = ex2_approx(y.y);
+        }
+        acc4[q & 3] = __fadd2_rn(acc4[q & 3], make_float2(s[2 * q], s[2 * q + 1]));
+      }
+      acc4[0] = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
+      l = alpha * l + (acc4[0].x + acc4[0].y);
+      // S * p (packed FMUL2), then the E4M3 cast, four keys per word
+      const float2 S2 = make_float2(S, S);
+      uint32_t pw[HC / 4];
+#pragma unroll
+      for (int q = 0; q < HC / 4; ++q) {
+        const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
+        const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
+        pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
+      }
+      if constexpr (COUNT) {
+        // Collapse: a visible non-sink key whose E4M3 byte is zero (P~ is never
+        // negative, so byte 0 <=> the cast flushed S*p to zero).
+        const bool all_valid = j0 >= p.n_sink && !need_mask;
+        const uint32_t cblk = zero_bytes<HC>(pw, k0, max(p.n_sink - j0, 0),
+                                             min(lim - j0, BN - 1), all_valid);
+        cnt += cblk;
+        if (j0 < p.n_sink) cnt_sink += cblk;
+      }
+      if (t > 0) {
+        // P~V(t-1) must be done: it reads the P~ tile and accumulates into O
+        ok = warp_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE);
+        if (!ok) break;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int q = 0; q < HC / 16; ++q) {
+        const uint32_t chunk = (uint32_t)(part * (HC / 16) + q);
+        const uint32_t dst = prow + ((chunk ^ pswz) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pw[4 * q]),
                      "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
                      : "memory");
       }
-      alpha_sm[(x * 2 + (t & 1)) * BM + r] = alpha;
-      if (t == T - 1) lsum_sm[x * BM + r] = l;
+      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o<OC>(tO, alpha);
       fence_proxy_async_smem();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.p_full(x, t & 1));
+      if (lane == 0) mbar_arrive(bar_p_full);
+    }
+
+    if (ok) ok = warp_wait(bar_o_done, (T - 1) & 1, ctl, WAIT_EPI_O_DONE);
+    if (ok) {
+      // the parts of a row add their row sums and counts
+      xl[part * BM + r] = l;
+      xcnt[part * BM + r] = cnt;
+      ok = pair_exchange(bar_fin(quarter), 0, ctl, lane);
     }
     if (ok) {
+      float lt = xl[r];
+      uint32_t ct = xcnt[r];
+#pragma unroll
+      for (int q = 1; q < NSPLIT; ++q) {
+        lt += xl[q * BM + r];
+        ct += xcnt[q * BM + r];
+      }
+      tc_fence_after();
+      const bool live = row < p.N;
+      store_row<OC, OUT_BF16>(tO, S * lt, live, p.O,
+                              ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D + part * OC);
       if constexpr (COUNT) {
-        const bool live = row < p.N;
         if (!live) cnt = cnt_sink = 0;   // padding rows past a ragged N
-        if (p.rows && live) p.rows[(size_t)bh * p.N + row] = cnt;
+        if (p.rows && live && part == 0) p.rows[(size_t)bh * p.N + row] = ct;
         const uint32_t wsum = __reduce_add_sync(0xffffffffu, cnt);
         const uint32_t wsink = __reduce_add_sync(0xffffffffu, cnt_sink);
         if (lane == 0) {
@@ -563,7 +545,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicCAS(p.status, 0u, 0x100u | *abort_flag);
-  if (warp == 13) {
+  if (warp == NSOFTMAX + 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
@@ -635,24 +617,14 @@ bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Registers per thread the kernel is compiled for.  Its warpgroups then move
-// registers among themselves with setmaxnreg (184 + 184 + 80 + 64 per thread,
-// x 128 threads each = 512 x 128); a launch with any other per-thread count
-// could leave the increase waiting forever, so it is refused.
-constexpr int LAUNCH_REGS = 128;
-
 template <int D, int BN, bool OUT_BF16, bool COUNT>
 cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                    const fp8attn::KParams& kp, cudaStream_t stream) {
   using L = fp8attn::Smem<D, BN>;
   auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT>;
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
-  if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
-  if (e != cudaSuccess) return e;
-  dim3 grid(kp.num_q_blocks, kp.B * kp.H);
+  dim3 grid(kp.num_q_tiles, kp.B * kp.H);
   kern<<<grid, fp8attn::NTHREADS, L::ALLOC, stream>>>(q, k, v, kp);
   return cudaGetLastError();
 }
@@ -699,8 +671,7 @@ const char* fp8attn_device_status_string(unsigned int word) {
     case fp8attn::WAIT_SM_S_FULL: return "timeout: softmax waiting for S";
     case fp8attn::WAIT_SM_O_DONE: return "timeout: softmax waiting for P~V";
     case fp8attn::WAIT_EPI_O_DONE: return "timeout: epilogue waiting for the last P~V";
-    case fp8attn::WAIT_CORR_P: return "timeout: correction waiting for the P~ tile";
-    case fp8attn::WAIT_CORR_O_DONE: return "timeout: correction waiting for P~V";
+    case 0x20: return "timeout: softmax waiting for the other part of its rows";
     default: return "timeout: unknown wait";
   }
 }
@@ -755,7 +726,7 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.causal = p->causal;
   kp.kv_order = p->kv_order;
   kp.n_sink = p->n_sink;
-  kp.num_q_blocks = (p->N + fp8attn::NTILE * fp8attn::BM - 1) / (fp8attn::NTILE * fp8attn::BM);
+  kp.num_q_tiles = (p->N + fp8attn::BM - 1) / fp8attn::BM;
   kp.scale_log2 = p->scale * fp8attn::LOG2E;
   kp.S = p->S;
   kp.O = p->O;
