@@ -44,9 +44,7 @@ namespace fp8attn {
 
 constexpr int BM = 128;         // query rows per CTA (= MMA M, = TMEM lanes)
 constexpr int NSTAGE = 2;       // K/V ring depth
-constexpr int NSPLIT = 2;       // softmax threads per query row (each owns block_n / 2 keys)
-constexpr int NSOFTMAX = 4 * NSPLIT;            // softmax warps
-constexpr int NTHREADS = 32 * (NSOFTMAX + 2);   // + TMA warp + MMA warp
+constexpr int NTHREADS = 192;   // 4 softmax warps + TMA warp + MMA warp
 constexpr float LOG2E = 1.4426950408889634f;
 // Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
 // (exp2_poly.cuh) and the rest on MUFU ex2: the two units then share the
@@ -71,6 +69,7 @@ enum : uint32_t {
 
 struct KParams {
   int B, H, Hkv, N, group;
+  float log2_S;       // log2(S) when S is an exact power of two (folded into the exponent)
   int causal, kv_order, n_sink;
   int num_q_tiles;
   float scale_log2;   // scale * log2(e)
@@ -90,13 +89,11 @@ struct Smem {
   static constexpr int K = Q + BM * D;
   static constexpr int V = K + NSTAGE * BN * D;
   static constexpr int P = V + NSTAGE * BN * D;
-  static constexpr int XMAX = P + BM * BN;                  // float [2 buffers][NSPLIT][BM]
-  static constexpr int XFIN = XMAX + 2 * NSPLIT * BM * 4;   // float l, uint count [NSPLIT][BM]
-  static constexpr int BAR = XFIN + 2 * NSPLIT * BM * 4;
+  static constexpr int BAR = P + BM * BN;
   // barriers: q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full, s_free, p_full,
-  // o_done, drain, xch[4 quarters][2 buffers], fin[4 quarters]
-  static constexpr int NBAR = 1 + 4 * NSTAGE + 5 + 4 * 2 + 4;
-  static constexpr int MISC = BAR + 8 * NBAR;   // tmem base slot, abort flag, drain flag
+  // o_done, drain
+  static constexpr int NBAR = 1 + 4 * NSTAGE + 5;
+  static constexpr int MISC = BAR + 8 * NBAR;   // tmem base slot, abort flag
   static constexpr int BYTES = MISC + 16;
   // slack to align the base to 1024, and at least 80 KB so that no more than two
   // CTAs share an SM: two 256-column TMEM allocations fill the SM's 512 columns
@@ -109,140 +106,19 @@ __device__ __forceinline__ int kv_block_at(int t, int T, int order) {
   return order == FP8ATTN_KV_FORWARD ? t : T - 1 - t;
 }
 
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
-                                          uint32_t where) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl, where));
-}
-
-// The NSPLIT softmax warps that share one TMEM lane quarter (the parts of the
-// same 32 rows) meet on an mbarrier of count NSPLIT: each warp publishes its
-// values in shared memory, arrives once, and waits (bounded, abort-aware) for
-// the others.
-__device__ __forceinline__ bool pair_exchange(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
-                                              int lane) {
-  __syncwarp();
-  if (lane == 0) mbar_arrive(bar);
-  return warp_wait(bar, parity, ctl, 0x20);
-}
-
-// Largest of n values, 8 independent chains then a tree.
-template <int N>
-__device__ __forceinline__ float row_max(const float (&s)[N]) {
-  float m8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-  for (int j = 8; j < N; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
-#pragma unroll
-  for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m8[i] = fmaxf(m8[i], m8[i + w]);
-  return m8[0];
-}
-
-// Number of zero bytes among the valid lanes of HC/4 packed E4M3 words
-// (collapse count of one part of a row).  Valid keys: block-local index in
-// [lo, hi]; all_valid skips the lane masks.  Four independent accumulators.
-template <int HC>
-__device__ __forceinline__ uint32_t zero_bytes(const uint32_t (&pw)[HC / 4], int k0, int lo, int hi,
-                                               bool all_valid) {
-  uint32_t z[4] = {0, 0, 0, 0};
-#pragma unroll
-  for (int q = 0; q < HC / 4; ++q) {
-    const uint32_t w = pw[q];
-    uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
-    if (!all_valid) {
-      const int a = lo - (k0 + 4 * q), bq = hi - (k0 + 4 * q);   // valid lanes a..bq of the word
-      const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
-      const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
-      y &= mlo & mhi;
-    }
-    z[q & 3] += y >> 7;   // one count per byte lane
-  }
-  const uint32_t zs = (z[0] + z[1]) + (z[2] + z[3]);   // byte lanes hold <= HC/4 each
-  return (zs * 0x01010101u) >> 24;
-}
-
-// O (NC TMEM columns of this warp's 32 rows) *= alpha, 32 columns per round trip.
-template <int NC>
-__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
-  const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-  for (int cc = 0; cc < NC / 32; ++cc) {
-    uint32_t o[32];
-    tmem_ld32(tO + 32 * cc, o);
-    tmem_wait_ld();
-#pragma unroll
-    for (int k = 0; k < 32; k += 2) {
-      const float2 r =
-          __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), a2);
-      o[k] = __float_as_uint(r.x);
-      o[k + 1] = __float_as_uint(r.y);
-    }
-    tmem_st32(tO + 32 * cc, o);
-  }
-  tmem_wait_st();
-}
-
-// Epilogue of one row part: NC columns of O / (S l) from TMEM to global memory
-// (BF16 RNE or FP32), 32 columns at a time, divided in place.
-template <int NC, bool OUT_BF16>
-__device__ __forceinline__ void store_row(uint32_t tO, float denom, bool live, void* O,
-                                          size_t obase) {
-#pragma unroll
-  for (int cc = 0; cc < NC / 32; ++cc) {
-    uint32_t o[32];
-    tmem_ld32(tO + 32 * cc, o);
-    tmem_wait_ld();
-#pragma unroll
-    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__fdiv_rn(__uint_as_float(o[k]), denom));
-    if (live) {
-      if constexpr (OUT_BF16) {
-        uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(O) + obase + 32 * cc);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
-                : "=r"(w[i])
-                : "f"(__uint_as_float(o[8 * k + 2 * i + 1])), "f"(__uint_as_float(o[8 * k + 2 * i])));
-          out[k] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      } else {
-        uint4* out = reinterpret_cast<uint4*>(static_cast<float*>(O) + obase + 32 * cc);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          out[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
-      }
-    }
-  }
-}
-
-// One CTA = one 128-row query tile of one (batch, head); two CTAs share an SM.
-//   warps 0-7  softmax: warp w holds rows 32(w%4)..+31 (its TMEM lane quarter)
-//              and keys [w/4 * BN/2, (w/4 + 1) * BN/2) of each KV block, and
-//              columns [w/4 * D/2, (w/4 + 1) * D/2) of O; the two warps of a
-//              quarter exchange their partial row maxima each block
-//   warp 8     TMA producer: Q tile once, K and V of each KV block in visiting
-//              order into a 2-stage ring, K one step ahead of V
-//   warp 9     MMA issuer and TMEM owner: S = Q K^T, O += P~ V
-// TMEM: S [0, BN), O [BN, BN + D).
-template <int D, int BN, bool OUT_BF16, bool COUNT>
+// FOLD: S is a power of two 2^k.  Then S * 2^(x - m) = 2^(x - m + k) exactly
+// (multiplying by 2^k only moves the exponent), so k joins the exponent's FMA
+// and the product disappears; the row sum is brought back by 2^-k, also exact.
+template <int D, int BN, bool OUT_BF16, bool COUNT, bool FOLD>
 __global__ void __launch_bounds__(NTHREADS, 2)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p) {
   using L = Smem<D, BN>;
-  constexpr int HC = BN / NSPLIT;   // keys per softmax thread
-  constexpr int OC = D / NSPLIT;    // O columns per softmax thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::Q, sK = sbase + L::K, sV = sbase + L::V, sP = sbase + L::P;
-  float* xmax = reinterpret_cast<float*>(smem + L::XMAX);
-  float* xl = reinterpret_cast<float*>(smem + L::XFIN);
-  uint32_t* xcnt = reinterpret_cast<uint32_t*>(smem + L::XFIN + NSPLIT * BM * 4);
   const uint32_t bar0 = sbase + L::BAR;
   const uint32_t bar_q_full = bar0;
   auto bar_k_full = [&](int s) { return bar0 + 8u * (1 + s); };
@@ -254,11 +130,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_o_done = bar_s_full + 24;
   const uint32_t bar_drain = bar_s_full + 32;
-  auto bar_xch = [&](int quarter, int buf) { return bar_s_full + 40 + 8u * (2 * quarter + buf); };
-  auto bar_fin = [&](int quarter) { return bar_s_full + 40 + 64 + 8u * quarter; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 4);
-  volatile uint32_t* never_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = p.causal ? (p.num_q_tiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
@@ -269,7 +142,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int last_row = min(q0 + BM - 1, p.N - 1);
   const int T = p.causal ? (last_row / BN + 1) : ((p.N + BN - 1) / BN);
   const WaitCtl ctl{abort_flag, p.timeout_ns};
-  const WaitCtl drain{never_flag, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
@@ -280,24 +152,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(bar_v_empty(s), 1);
     }
     mbar_init(bar_s_full, 1);
-    mbar_init(bar_s_free, NSOFTMAX);
-    mbar_init(bar_p_full, NSOFTMAX);
+    mbar_init(bar_s_free, 4);
+    mbar_init(bar_p_full, 4);
     mbar_init(bar_o_done, 1);
     mbar_init(bar_drain, 1);
-    for (int qd = 0; qd < 4; ++qd) {
-      mbar_init(bar_xch(qd, 0), NSPLIT);
-      mbar_init(bar_xch(qd, 1), NSPLIT);
-      mbar_init(bar_fin(qd), NSPLIT);
-    }
     *abort_flag = 0;
-    *never_flag = 0;
+    *reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8) = 0;   // never raised: drain waits
     fence_barrier_init();
   }
-  if (warp == NSOFTMAX + 1) {
+  if (warp == 5) {
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == NSOFTMAX && lane == 0) {
+  if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -307,7 +174,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == NSOFTMAX) {
+  if (warp == 4) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q_full, BM * D);
@@ -337,15 +204,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     bkv);
         v_issued = t + 1;
       }
-      // drain: the last load issued into each stage must land before the CTA
-      // exits (immediate when the consumers took them all; needed after an abort)
-      for (int t = k_issued - 1; t >= 0 && t >= k_issued - NSTAGE; --t)
-        mbar_wait(bar_k_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
-      for (int t = v_issued - 1; t >= 0 && t >= v_issued - NSTAGE; --t)
-        mbar_wait(bar_v_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
-      mbar_wait(bar_q_full, 0, drain, 0);
+      {
+        // drain: the last load issued into each stage must land before the CTA
+        // exits (immediate when the consumers took them all; needed after an abort)
+        const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8),
+                            p.timeout_ns};
+        for (int t = k_issued - 1; t >= 0 && t >= k_issued - NSTAGE; --t)
+          mbar_wait(bar_k_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
+        for (int t = v_issued - 1; t >= 0 && t >= v_issued - NSTAGE; --t)
+          mbar_wait(bar_v_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
+        mbar_wait(bar_q_full, 0, drain, 0);
+      }
     }
-  } else if (warp == NSOFTMAX + 1) {
+  } else if (warp == 5) {
     // ----------------------------------------------------------------- MMA --
     constexpr uint32_t SWZ_QK = (D == 128) ? SWZ_128B : SWZ_64B;
     constexpr uint32_t SWZ_P = (BN == 128) ? SWZ_128B : SWZ_64B;
@@ -386,7 +257,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int kk = 0; kk < BN / 32; ++kk) {
           const uint64_t a = smem_desc(sP + 32 * kk, 16, 8 * BN, SWZ_P);
-          const uint64_t bdesc = smem_desc(sV + st * BN * D + kk * 32 * D, BN * D, 8 * D, SWZ_QK);
+          const uint64_t bdesc =
+              smem_desc(sV + st * BN * D + kk * 32 * D, BN * D, 8 * D, SWZ_QK);
           mma_e4m3_ss(tO, a, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar_o_done);
@@ -394,70 +266,79 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       __syncwarp();
     }
-    // drain every MMA this warp issued before TMEM is released
-    if (lane == 0) mma_commit(bar_drain);
-    __syncwarp();
-    mbar_wait(bar_drain, 0, drain, 0);
+    if (!ok) {
+      // drain every MMA this warp issued before TMEM is released
+      const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8), p.timeout_ns};
+      if (lane == 0) mma_commit(bar_drain);
+      __syncwarp();
+      mbar_wait(bar_drain, 0, drain, 0);
+    }
   } else {
     // ------------------------------------------------------------- softmax --
-    const int quarter = warp & 3, part = warp >> 2;
-    const int r = 32 * quarter + lane;            // row within the tile
+    const int r = threadIdx.x;   // row within the tile; warp w reads TMEM lanes 32w..32w+31
     const int row = q0 + r;
-    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const uint32_t tS = tmem_base + lane_off + part * HC;
-    const uint32_t tO = tmem_base + lane_off + BN + part * OC;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t tS = tmem_base + lane_off, tO = tmem_base + lane_off + BN;
     const float c = p.scale_log2;
     const float S = p.S;
+    const float inv_S = 1.f / S;   // exact when FOLD (S a power of two)
     float m_run = -INFINITY, l = 0.f;
     uint32_t cnt = 0, cnt_sink = 0;
     bool ok = true;
-    // this thread's part of the P~ row in the swizzled tile (128B swizzle for
-    // 128-byte rows, 64B swizzle for 64-byte rows)
+    // this thread's P~ row in the swizzled tile (128B swizzle for 128-byte rows,
+    // 64B swizzle for 64-byte rows)
     const uint32_t prow = sP + (r >> 3) * (8 * BN) + (r & 7) * BN;
     const uint32_t pswz = (BN == 128) ? (uint32_t)(r & 7) : (uint32_t)((r & 7) >> 1);
-    const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
-    const int k0 = part * HC;                                  // first key of this part
 
     for (int t = 0; t < T; ++t) {
       const int j0 = kv_block_at(t, T, p.kv_order) * BN;
-      ok = warp_wait(bar_s_full, t & 1, ctl, WAIT_SM_S_FULL);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, t & 1, ctl, WAIT_SM_S_FULL));
       if (!ok) break;
       tc_fence_after();
-      float s[HC];
+      uint32_t sr[BN];
 #pragma unroll
-      for (int cc = 0; cc < HC / 32; ++cc)
-        tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * cc]));
+      for (int cc = 0; cc < BN / 32; ++cc)
+        tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_s_free);
 
+      float* s = reinterpret_cast<float*>(sr);
       const bool need_mask = (p.causal && j0 + BN - 1 > q0) || (j0 + BN > p.N);
+      const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
       if (need_mask) {
 #pragma unroll
-        for (int j = 0; j < HC; ++j)
-          if (j0 + k0 + j > lim) s[j] = -INFINITY;
+        for (int j = 0; j < BN; ++j)
+          if (j0 + j > lim) s[j] = -INFINITY;
       }
-      // row max: this part's, then the partner's through shared memory
-      float* xm = xmax + (t & 1) * NSPLIT * BM;
-      xm[part * BM + r] = row_max<HC>(s);
-      ok = pair_exchange(bar_xch(quarter, t & 1), (t >> 1) & 1, ctl, lane);
-      if (!ok) break;
-      float mx = xm[r];
+      // row max: 16 independent chains of three-input max, then a tree
+      float mx16[16];
 #pragma unroll
-      for (int q = 1; q < NSPLIT; ++q) mx = fmaxf(mx, xm[q * BM + r]);
+      for (int i = 0; i < 16; ++i) mx16[i] = s[i];
+#pragma unroll
+      for (int j = 16; j + 16 < BN; j += 32)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
+      if constexpr ((BN - 16) % 32 != 0) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
+      }
+      float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
+                       fmax3(mx16[6], mx16[7], mx16[8]));
+      mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
+      mx = fmaxf(mx, mx16[15]);
       const float m_new = fmaxf(m_run, mx * c);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-      m_run = m_new;
-      // p = 2^(s*c - m): packed FFMA2 for the argument, then MUFU ex2 (or the
-      // FMA-pipe polynomial for POLY_OF_8 of every 8 pairs), split packed row sums
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
-      float2 acc4[4];
+      // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
+      const float off = FOLD ? p.log2_S - m_use : -m_use;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(off, off);
+      float2 acc8[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc4[i] = make_float2(0.f, 0.f);
+      for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int q = 0; q < HC / 2; ++q) {
+      for (int q = 0; q < BN / 2; ++q) {
         const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
         if ((q & 7) < POLY_OF_8) {
           const float2 e = exp2_poly2(y);
@@ -467,71 +348,146 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           s[2 * q] = ex2_approx(y.x);
           s[2 * q + 1] = ex2_approx(y.y);
         }
-        acc4[q & 3] = __fadd2_rn(acc4[q & 3], make_float2(s[2 * q], s[2 * q + 1]));
+        acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
       }
-      acc4[0] = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
-      l = alpha * l + (acc4[0].x + acc4[0].y);
-      // S * p (packed FMUL2), then the E4M3 cast, four keys per word
-      const float2 S2 = make_float2(S, S);
-      uint32_t pw[HC / 4];
 #pragma unroll
-      for (int q = 0; q < HC / 4; ++q) {
-        const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
-        const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
-        pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
+      const float rowsum = acc8[0].x + acc8[0].y;
+      l = alpha * l + (FOLD ? rowsum * inv_S : rowsum);
+      // S * p (already in s[] when FOLD; else packed FMUL2), then the E4M3 cast,
+      // four keys per word
+      uint32_t pw[BN / 4];
+      if constexpr (FOLD) {
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q)
+          pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+      } else {
+        const float2 S2 = make_float2(S, S);
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+          const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
+          const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
+          pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
+        }
       }
       if constexpr (COUNT) {
-        // Collapse: a visible non-sink key whose E4M3 byte is zero (P~ is never
-        // negative, so byte 0 <=> the cast flushed S*p to zero).
-        const bool all_valid = j0 >= p.n_sink && !need_mask;
-        const uint32_t cblk = zero_bytes<HC>(pw, k0, max(p.n_sink - j0, 0),
-                                             min(lim - j0, BN - 1), all_valid);
+        // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
+        // negative, so byte 0 <=> the cast flushed S*p to zero.  Zero bytes are
+        // found four at a time; blocks that hold a sink or a masked key restrict
+        // the count to the lanes with n_sink <= j <= last visible key.
+        uint32_t zacc = 0;
+        if (j0 >= p.n_sink && !need_mask) {
+#pragma unroll
+          uint32_t z4[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int q = 0; q < BN / 4; ++q) {
+            const uint32_t w = pw[q];
+            z4[q & 3] += ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu) >> 7;
+          }
+          zacc = (z4[0] + z4[1]) + (z4[2] + z4[3]);
+        } else {
+          const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);   // block-local
+#pragma unroll
+          for (int q = 0; q < BN / 4; ++q) {
+            const uint32_t w = pw[q];
+            uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
+            const int a = lo - 4 * q, bq = hi - 4 * q;   // lanes a..bq of this word are valid
+            const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
+            const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
+            zacc += (y & mlo & mhi) >> 7;
+          }
+        }
+        const uint32_t cblk = (zacc * 0x01010101u) >> 24;   // byte lanes hold <= BN/4 each
         cnt += cblk;
         if (j0 < p.n_sink) cnt_sink += cblk;
       }
       if (t > 0) {
         // P~V(t-1) must be done: it reads the P~ tile and accumulates into O
-        ok = warp_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE));
         if (!ok) break;
         tc_fence_after();
       }
 #pragma unroll
-      for (int q = 0; q < HC / 16; ++q) {
-        const uint32_t chunk = (uint32_t)(part * (HC / 16) + q);
-        const uint32_t dst = prow + ((chunk ^ pswz) << 4);
+      for (int q = 0; q < BN / 16; ++q) {
+        const uint32_t dst = prow + ((q ^ pswz) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pw[4 * q]),
                      "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
                      : "memory");
       }
-      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o<OC>(tO, alpha);
+      if (t > 0) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          // O *= alpha for this warp's 32 rows, 64 TMEM columns per round trip
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; cc += 2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tO + 32 * cc, o0);
+            tmem_ld32(tO + 32 * cc + 32, o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              float2 r0 = __fmul2_rn(make_float2(__uint_as_float(o0[k]), __uint_as_float(o0[k + 1])), a2);
+              float2 r1 = __fmul2_rn(make_float2(__uint_as_float(o1[k]), __uint_as_float(o1[k + 1])), a2);
+              o0[k] = __float_as_uint(r0.x);
+              o0[k + 1] = __float_as_uint(r0.y);
+              o1[k] = __float_as_uint(r1.x);
+              o1[k + 1] = __float_as_uint(r1.y);
+            }
+            tmem_st32(tO + 32 * cc, o0);
+            tmem_st32(tO + 32 * cc + 32, o1);
+          }
+          tmem_wait_st();
+        }
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p_full);
+      m_run = m_new;
     }
 
-    if (ok) ok = warp_wait(bar_o_done, (T - 1) & 1, ctl, WAIT_EPI_O_DONE);
     if (ok) {
-      // the parts of a row add their row sums and counts
-      xl[part * BM + r] = l;
-      xcnt[part * BM + r] = cnt;
-      ok = pair_exchange(bar_fin(quarter), 0, ctl, lane);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (T - 1) & 1, ctl, WAIT_EPI_O_DONE));
     }
     if (ok) {
-      float lt = xl[r];
-      uint32_t ct = xcnt[r];
-#pragma unroll
-      for (int q = 1; q < NSPLIT; ++q) {
-        lt += xl[q * BM + r];
-        ct += xcnt[q * BM + r];
-      }
       tc_fence_after();
+      const float denom = S * l;
       const bool live = row < p.N;
-      store_row<OC, OUT_BF16>(tO, S * lt, live, p.O,
-                              ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D + part * OC);
+      const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * cc, o);
+        tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), denom);
+        if (live) {
+          if constexpr (OUT_BF16) {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              uint32_t bits;
+              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(bits) : "f"(v[2 * k + 1]), "f"(v[2 * k]));
+              w[k] = bits;
+            }
+            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + obase + 32 * cc);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              out[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          } else {
+            float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.O) + obase + 32 * cc);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              out[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
+        }
+      }
       if constexpr (COUNT) {
         if (!live) cnt = cnt_sink = 0;   // padding rows past a ragged N
-        if (p.rows && live && part == 0) p.rows[(size_t)bh * p.N + row] = ct;
+        if (p.rows && live) p.rows[(size_t)bh * p.N + row] = cnt;
         const uint32_t wsum = __reduce_add_sync(0xffffffffu, cnt);
         const uint32_t wsink = __reduce_add_sync(0xffffffffu, cnt_sink);
         if (lane == 0) {
@@ -545,7 +501,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicCAS(p.status, 0u, 0x100u | *abort_flag);
-  if (warp == NSOFTMAX + 1) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
@@ -617,11 +573,11 @@ bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D, int BN, bool OUT_BF16, bool COUNT>
+template <int D, int BN, bool OUT_BF16, bool COUNT, bool FOLD>
 cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                    const fp8attn::KParams& kp, cudaStream_t stream) {
   using L = fp8attn::Smem<D, BN>;
-  auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT>;
+  auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT, FOLD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(kp.num_q_tiles, kp.B * kp.H);
@@ -629,13 +585,28 @@ cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap
   return cudaGetLastError();
 }
 
+template <int D, int BN, bool FOLD>
+cudaError_t launch_f(bool bf16, bool count, const CUtensorMap& q, const CUtensorMap& k,
+                     const CUtensorMap& v, const fp8attn::KParams& kp, cudaStream_t s) {
+  if (bf16) return count ? launch<D, BN, true, true, FOLD>(q, k, v, kp, s)
+                         : launch<D, BN, true, false, FOLD>(q, k, v, kp, s);
+  return count ? launch<D, BN, false, true, FOLD>(q, k, v, kp, s)
+               : launch<D, BN, false, false, FOLD>(q, k, v, kp, s);
+}
+
 template <int D, int BN>
-cudaError_t launch_dt(bool bf16, bool count, const CUtensorMap& q, const CUtensorMap& k,
+cudaError_t launch_dt(bool bf16, bool count, bool fold, const CUtensorMap& q, const CUtensorMap& k,
                       const CUtensorMap& v, const fp8attn::KParams& kp, cudaStream_t s) {
-  if (bf16) return count ? launch<D, BN, true, true>(q, k, v, kp, s)
-                         : launch<D, BN, true, false>(q, k, v, kp, s);
-  return count ? launch<D, BN, false, true>(q, k, v, kp, s)
-               : launch<D, BN, false, false>(q, k, v, kp, s);
+  return fold ? launch_f<D, BN, true>(bf16, count, q, k, v, kp, s)
+              : launch_f<D, BN, false>(bf16, count, q, k, v, kp, s);
+}
+
+// log2(S) when S is an exact power of two with 2^k and 2^-k both normal, else NaN.
+float pow2_log2(float S) {
+  int e;
+  const float m = std::frexp(S, &e);
+  if (m != 0.5f || e - 1 < -125 || e - 1 > 125) return NAN;
+  return (float)(e - 1);
 }
 
 }  // namespace
@@ -671,7 +642,6 @@ const char* fp8attn_device_status_string(unsigned int word) {
     case fp8attn::WAIT_SM_S_FULL: return "timeout: softmax waiting for S";
     case fp8attn::WAIT_SM_O_DONE: return "timeout: softmax waiting for P~V";
     case fp8attn::WAIT_EPI_O_DONE: return "timeout: epilogue waiting for the last P~V";
-    case 0x20: return "timeout: softmax waiting for the other part of its rows";
     default: return "timeout: unknown wait";
   }
 }
@@ -740,14 +710,17 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
 
   const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;
   const bool count = p->collapse_ctr != nullptr;
+  const float k2 = pow2_log2(p->S);
+  const bool fold = !std::isnan(k2);
+  kp.log2_S = fold ? k2 : 0.f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (p->d == 128)
-    e = (bn == 128) ? launch_dt<128, 128>(bf16, count, mq, mk, mv, kp, s)
-                    : launch_dt<128, 64>(bf16, count, mq, mk, mv, kp, s);
+    e = (bn == 128) ? launch_dt<128, 128>(bf16, count, fold, mq, mk, mv, kp, s)
+                    : launch_dt<128, 64>(bf16, count, fold, mq, mk, mv, kp, s);
   else
-    e = (bn == 128) ? launch_dt<64, 128>(bf16, count, mq, mk, mv, kp, s)
-                    : launch_dt<64, 64>(bf16, count, mq, mk, mv, kp, s);
+    e = (bn == 128) ? launch_dt<64, 128>(bf16, count, fold, mq, mk, mv, kp, s)
+                    : launch_dt<64, 64>(bf16, count, fold, mq, mk, mv, kp, s);
   if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return FP8ATTN_OK;
 }
