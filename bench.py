@@ -91,6 +91,35 @@ def peak_tflops():
         return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2"
 
 
+KERNEL_SOURCES = ["online_softmax_tcgen05_b200/csrc/fp8_attn_fwd.cu",
+                  "online_softmax_tcgen05_b200/csrc/sm100.cuh",
+                  "online_softmax_tcgen05_b200/csrc/exp2_poly.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_prefill_N32768.json")
+
+
+def kernel_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+    the committed ncu capture of this workload, or None when the kernel sources
+    changed since that capture."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        if rec.get("kernel_sources_sha256") != kernel_sources_sha256():
+            return None
+        return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
+    except Exception:
+        return None
+
+
 def smi_index(local_rank):
     """nvidia-smi index of this process's GPU (CUDA_VISIBLE_DEVICES aware)."""
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
@@ -259,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
                             "nominal_4500": round(kernel_tflops / 4500.0, 4)},
         "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2),
                      "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(kernel_tflops / peak, 4), "traffic": None,
+                     "frac": round(kernel_tflops / peak, 4), "traffic": measured_traffic(),
                      "peak_source": peak_src + " (of measured)" if "measured" in peak_src
                      else peak_src},
         "collapse": {"fraction": frac, "count_per_step": collapse_total // args.steps // world,

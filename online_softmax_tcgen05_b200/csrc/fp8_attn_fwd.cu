@@ -379,7 +379,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // the count to the lanes with n_sink <= j <= last visible key.
         uint32_t zacc = 0;
         if (j0 >= p.n_sink && !need_mask) {
-#pragma unroll
           uint32_t z4[4] = {0, 0, 0, 0};
 #pragma unroll
           for (int q = 0; q < BN / 4; ++q) {
