@@ -57,6 +57,11 @@ typedef enum {
 
 enum { FP8ATTN_KV_FORWARD = 0, FP8ATTN_KV_REVERSE = 1 };
 enum { FP8ATTN_O_BF16 = 0, FP8ATTN_O_F32 = 1 };
+/* Row-sum (denominator) source.  FP32_P: l from the FP32 P before the cast and
+ * O = acc / (S l) (the P-cast paper's kernel).  CAST_P: l from the cast values,
+ * l = sum_j dec(pt_j), and O = acc / l, so numerator and denominator use the same
+ * quantised operand (the choice EFQ-Softmax makes). */
+enum { FP8ATTN_DENOM_FP32_P = 0, FP8ATTN_DENOM_CAST_P = 1 };
 
 /* fp8_attn_fwd - the attention forward above, square self-attention, H_kv = H,
  * O in BF16, KV block 128.
@@ -93,6 +98,9 @@ typedef struct {
   int o_dtype;            /* FP8ATTN_O_BF16 (RNE) or FP8ATTN_O_F32 */
   int block_n;            /* KV block: 0 (= 128), 64 or 128.  N need not be a multiple:
                              the last block then holds the remaining keys. */
+  int denominator;        /* FP8ATTN_DENOM_FP32_P (default, 0) or FP8ATTN_DENOM_CAST_P;
+                             CAST_P needs S >= 2^-8 so that the row maximum's cast is
+                             nonzero */
   unsigned long long* collapse_ctr;      /* nullable; += all collapsed entries */
   unsigned long long* collapse_sink_ctr; /* nullable; += those in KV blocks holding a
                                             sink key (requires collapse_ctr) */

@@ -17,15 +17,16 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass
 
-from ._binding import (ECUDA, EINVAL, ETIMEOUT, EUNSUPPORTED, KV_FORWARD, KV_REVERSE, O_BF16,
-                       O_F32, OK, Fp8AttnError, device_status_string, fp8_attn_fwd,
+from ._binding import (DENOM_CAST_P, DENOM_FP32_P, ECUDA, EINVAL, ETIMEOUT, EUNSUPPORTED,
+                       KV_FORWARD, KV_REVERSE, O_BF16, O_F32, OK, Fp8AttnError, device_status_string, fp8_attn_fwd,
                        fp8_attn_fwd_ex, fp8_e4m3_scale_cast, last_error, load_library,
                        status_string)
 
 __all__ = ["attention", "AttentionStats", "fp8_attn_fwd", "fp8_attn_fwd_ex",
            "fp8_e4m3_scale_cast", "load_library", "status_string", "last_error",
            "device_status_string", "Fp8AttnError", "KV_FORWARD", "KV_REVERSE", "O_BF16",
-           "O_F32", "OK", "EINVAL", "EUNSUPPORTED", "ECUDA", "ETIMEOUT", "e4m3_cast"]
+           "O_F32", "OK", "EINVAL", "EUNSUPPORTED", "ECUDA", "ETIMEOUT", "e4m3_cast",
+           "DENOM_FP32_P", "DENOM_CAST_P"]
 
 
 @dataclass
@@ -54,6 +55,7 @@ def e4m3_cast(x, S: float = 1.0):
 
 def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: float = 256.0,
               kv_order: int = KV_REVERSE, n_sink: int = 0, block_n: int = 0,
+              denominator: int = DENOM_FP32_P,
               out_dtype=None, count_collapse: bool = False, per_row: bool = False,
               out=None, stream=None):
     """FP8 attention forward.  Returns (O, AttentionStats)."""
@@ -80,6 +82,7 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     fp8_attn_fwd_ex(q, k, v, o, B=B, H=H, H_kv=H_kv, N=N, d=d, causal=causal,
                     scale=scale if scale is not None else 1.0 / math.sqrt(d), S=S,
                     kv_order=kv_order, n_sink=n_sink, o_dtype=o_code, block_n=block_n,
+                    denominator=denominator,
                     collapse_ctr=None if ctr is None else ctr[0:1],
                     collapse_sink_ctr=None if ctr is None else ctr[1:2],
                     collapse_rows=rows, stream=stream)

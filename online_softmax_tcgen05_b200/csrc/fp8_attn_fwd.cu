@@ -81,6 +81,7 @@ struct KParams {
   unsigned int* status;
   unsigned long long timeout_ns;
   int debug_skip_kv_step;   // testing hook: 1-based KV step whose K load is never issued
+  int denom_cast;           // row sum from the cast values (FP8ATTN_DENOM_CAST_P)
 };
 
 template <int D, int BN>
@@ -355,7 +356,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
       const float rowsum = acc8[0].x + acc8[0].y;
-      l = alpha * l + (FOLD ? rowsum * inv_S : rowsum);
+      if (!p.denom_cast) l = alpha * l + (FOLD ? rowsum * inv_S : rowsum);
       // S * p (already in s[] when FOLD; else packed FMUL2), then the E4M3 cast,
       // four keys per word
       uint32_t pw[BN / 4];
@@ -371,6 +372,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
           pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
         }
+      }
+      if (p.denom_cast) {
+        // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
+        // form a float exactly 2^-120 times the E4M3 value (subnormals included,
+        // as FP32 subnormals); sum those, then scale by 2^120 (exact).
+        float2 d4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d4[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+          const uint32_t w = pw[q];
+          const float2 lo = make_float2(__uint_as_float((w & 0x7Fu) << 20),
+                                        __uint_as_float((w & 0x7F00u) << 12));
+          const float2 hi = make_float2(__uint_as_float((w & 0x7F0000u) << 4),
+                                        __uint_as_float((w & 0x7F000000u) >> 4));
+          d4[q & 3] = __fadd2_rn(d4[q & 3], __fadd2_rn(lo, hi));
+        }
+        d4[0] = __fadd2_rn(__fadd2_rn(d4[0], d4[1]), __fadd2_rn(d4[2], d4[3]));
+        l = alpha * l + (d4[0].x + d4[0].y) * 0x1p120f;
       }
       if constexpr (COUNT) {
         // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
@@ -452,7 +472,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     if (ok) {
       tc_fence_after();
-      const float denom = S * l;
+      const float denom = p.denom_cast ? l : S * l;
       const bool live = row < p.N;
       const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
 #pragma unroll
@@ -661,6 +681,10 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   if (p->kv_order != FP8ATTN_KV_FORWARD && p->kv_order != FP8ATTN_KV_REVERSE)
     return fail(FP8ATTN_EINVAL, "kv_order must be 0 (forward) or 1 (reverse)");
   if (p->n_sink < 0 || p->n_sink > p->N) return fail(FP8ATTN_EINVAL, "n_sink must be in [0, N]");
+  if (p->denominator != FP8ATTN_DENOM_FP32_P && p->denominator != FP8ATTN_DENOM_CAST_P)
+    return fail(FP8ATTN_EINVAL, "denominator must be FP8ATTN_DENOM_FP32_P or FP8ATTN_DENOM_CAST_P");
+  if (p->denominator == FP8ATTN_DENOM_CAST_P && std::isfinite(p->S) && p->S < 0x1p-8f)
+    return fail(FP8ATTN_EINVAL, "the cast-value denominator needs S >= 2^-8");
   if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
     return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
   if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
@@ -705,6 +729,7 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.status = p->status_word;
   kp.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
   kp.debug_skip_kv_step = p->debug_skip_kv_step;
+  kp.denom_cast = p->denominator == FP8ATTN_DENOM_CAST_P;
   if (kp.B * kp.H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
 
   const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;

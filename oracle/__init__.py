@@ -66,7 +66,7 @@ def lib():
         L.oracle_attn_exact.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, i64, P, i32]
         L.oracle_attn_exact.restype = i32
         L.oracle_attn_emulate.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f32, f32,
-                                          i32, i32, i32, i32, P, i64, P, P, P, i32]
+                                          i32, i32, i32, i32, P, i64, P, P, P, i32, i32]
         L.oracle_attn_emulate.restype = i32
         L.oracle_collapse_logits.argtypes = [P, i64, i32, i32, i32, f32, i32, P, P, i32]
         L.oracle_collapse_logits.restype = i32
@@ -131,9 +131,11 @@ def attn_exact(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, rows=None, nthreads=0
 
 
 def attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, kv_order, block_n, n_sink,
-                 o_bf16=False, rows=None, nthreads=0):
+                 o_bf16=False, rows=None, nthreads=0, denom_mode=0):
     """FP8 pipeline emulation.  Returns (O [nrows, d] float32, collapse per row
-    uint32, totals uint64[2] = {in sink-holding KV blocks, in other blocks})."""
+    uint32, totals uint64[2] = {in sink-holding KV blocks, in other blocks}).
+    denom_mode 0: l from the FP32 P, O = acc / (S l); 1: l from the cast values,
+    O = acc / l."""
     for a in (Q8, K8, V8):
         assert a.dtype == np.uint8 and a.flags.c_contiguous
     r, nr = _rows(rows)
@@ -144,7 +146,7 @@ def attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, kv_order, block_
     rc = lib().oracle_attn_emulate(_ptr(Q8), _ptr(K8), _ptr(V8), B, H, Hkv, N, d, int(causal),
                                    float(scale), float(S), int(kv_order), int(block_n),
                                    int(n_sink), int(bool(o_bf16)), _ptr(r), nr, _ptr(O),
-                                   _ptr(cr), _ptr(tot), nthreads)
+                                   _ptr(cr), _ptr(tot), nthreads, int(denom_mode))
     if rc:
         raise ValueError("oracle_attn_emulate: bad shape")
     return O, cr, tot

@@ -230,6 +230,8 @@ int oracle_attn_exact(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
 //     acc_k  = alpha * acc_k + sum_j dec(pt_j) * dec(v_jk)   (j ascending)
 //     m = m'
 //   O_k = acc_k / fl32(S * l), then BF16 RNE when o_bf16.
+// denom_mode 1 (the denominator from the quantised operand, as EFQ-Softmax
+// does): l = alpha * l + sum_j dec(pt_j)  (j ascending) and O_k = acc_k / l.
 // Outputs: O [nrows, d] (float), collapse_rows [nrows] (nullable),
 // collapse_totals[2] = {entries in KV blocks holding a sink key, entries in the
 // other blocks} (nullable, accumulated).
@@ -238,7 +240,7 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
                         int kv_order, int block_n, int n_sink, int o_bf16,
                         const int64_t* rows, int64_t nrows,
                         float* O, uint32_t* collapse_rows, uint64_t* collapse_totals,
-                        int nthreads) {
+                        int nthreads, int denom_mode) {
     if (H % Hkv || block_n <= 0) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
@@ -260,6 +262,7 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
             for (int k = 0; k < d; ++k) q[k] = g_dec[qp[k]];
             for (int k = 0; k < d; ++k) acc[k] = 0.0f;
             RowState st;
+            float lq = 0.0f;   // denominator from the cast values (denom_mode 1)
             uint32_t row_collapse = 0;
             const int last = causal ? i / block_n : nblocks - 1;
             for (int step = 0; step <= last; ++step) {
@@ -279,6 +282,9 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
                 row_collapse += (uint32_t)c;
                 if (block_has_sink(blk, block_n, n_sink)) tot_sink += (uint64_t)c;
                 else tot_other += (uint64_t)c;
+                float qsum = 0.0f;
+                for (int jj = 0; jj < nb; ++jj) qsum += g_dec[pt[jj]];
+                lq = alpha * lq + qsum;
                 for (int k = 0; k < d; ++k) acc[k] = alpha * acc[k];
                 for (int jj = 0; jj < nb; ++jj) {
                     float pv = g_dec[pt[jj]];
@@ -287,7 +293,7 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
                     for (int k = 0; k < d; ++k) acc[k] += pv * g_dec[vp[k]];
                 }
             }
-            float denom = S * st.l;
+            float denom = denom_mode ? lq : S * st.l;
             for (int k = 0; k < d; ++k) {
                 float o = acc[k] / denom;
                 O[t * d + k] = o_bf16 ? bf16_rne(o) : o;

@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 
 def run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, n_sink, f32=True, scale=None,
-            count=True):
+            count=True, denominator=0):
     import torch
     from online_softmax_tcgen05_b200 import O_BF16, O_F32, fp8_attn_fwd_ex
     (Qg, _), (Kg, _), (Vg, _) = ins
@@ -37,7 +37,8 @@ def run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, n_sink, f32=True, s
     fp8_attn_fwd_ex(Qg, Kg, Vg, O, B=B, H=H, H_kv=Hkv, N=N, d=d, causal=causal,
                     scale=scale if scale is not None else 1.0 / math.sqrt(d), S=S,
                     kv_order=order, n_sink=n_sink, o_dtype=O_F32 if f32 else O_BF16,
-                    block_n=block_n, collapse_ctr=ctr[0:1] if count else None,
+                    block_n=block_n, denominator=denominator,
+                    collapse_ctr=ctr[0:1] if count else None,
                     collapse_sink_ctr=ctr[1:2] if count else None,
                     collapse_rows=rows if count else None, status_word=status)
     torch.cuda.synchronize()
@@ -273,3 +274,40 @@ def test_long_context_full_size():
                                        128, o_bf16=True, rows=hit)
         assert np.abs(cr.astype(np.int64) - out_rows[hit]).sum() <= 1, (hit, cr, out_rows[hit])
     check_case(W, ins, 1, 1.0, 0, 128, f32=False, rows=rows[::3], what="long fwd 1")
+
+
+def test_mse_gain_grows_with_sequence_length_on_gpu():
+    """The paper's sequence-length claim on the kernel's own outputs: the MSE
+    (against float64 attention on the same E4M3 inputs) of forward S = 1 over
+    reverse S = 256 grows with N, from 1k to 128k keys."""
+    gains = []
+    for N in (1024, 4096, 16384, 65536, 131072):
+        B, H, d = 1, 2, 128
+        W = workload.make_sink_workload(B, H, H, N, d, 4, 7.0, seed=workload.CONFIG_SEED_BASE + 6)
+        ins = gpu_inputs(W)
+        (_, Q8), (_, K8), (_, V8) = ins
+        rows = sample_rows(B, H, N, 128, seed=9)
+        ref = oracle.attn_exact(Q8, K8, V8, B, H, H, N, d, 0, W.scale, rows=rows)
+        mse = {}
+        for order, S in ((0, 1.0), (1, 256.0)):
+            Og, *_ = run_gpu(ins, B, H, H, N, d, 0, S, order, 128, 4)
+            mse[(order, S)] = float(np.mean((Og[rows] - ref) ** 2))
+        gains.append(mse[(0, 1.0)] / mse[(1, 256.0)])
+    assert all(a < b for a, b in zip(gains, gains[1:])), gains
+    assert gains[-1] > 4 * gains[0], gains
+
+
+
+@pytest.mark.parametrize("B,H,Hkv,N,d,block_n,causal", [(1, 2, 1, 700, 128, 128, 1),
+                                                        (1, 2, 2, 520, 64, 64, 0)])
+def test_cast_denominator_parity(B, H, Hkv, N, d, block_n, causal):
+    """Row sum from the cast values (FP8ATTN_DENOM_CAST_P) against the oracle."""
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 9.0, seed=60 + N)
+    ins = gpu_inputs(W)
+    (_, Q8), (_, K8), (_, V8) = ins
+    for S in (1.0, 256.0, 448.0):
+        for order in (0, 1):
+            Og, *_ = run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, 4, denominator=1)
+            Oe, _, _ = oracle.attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, W.scale, S, order,
+                                           block_n, 4, denom_mode=1)
+            assert_o_close(Og, Oe, ("cast denominator", S, order))
