@@ -384,8 +384,9 @@ def test_cast_denominator_matches_brute_force(oracle_mod, N, d, block_n, causal)
 
 def test_cast_denominator_weights_sum_to_one(oracle_mod):
     """With numerator and denominator from the same cast values the weights sum
-    to one: constant V = 2^k comes out exactly 2^k, collapse or not; the FP32-P
-    denominator instead keeps the collapsed mass and shrinks O."""
+    to one: constant V = 2^k comes out 2^k up to the FP32 summation order (the
+    numerator adds key by key, the denominator block sums), collapse or not; the
+    FP32-P denominator instead keeps the collapsed mass and shrinks O."""
     B, H, N, d = 1, 1, 512, 32
     W = workload.make_sink_workload(B, H, H, N, d, 4, 10.0, seed=41)
     Q8, K8 = oracle_mod.e4m3_encode(W.q), oracle_mod.e4m3_encode(W.k)
@@ -393,7 +394,7 @@ def test_cast_denominator_weights_sum_to_one(oracle_mod):
     for S, order in ((1.0, 0), (256.0, 1), (448.0, 0)):
         O1, cr, _ = oracle_mod.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, W.scale, S, order, 128, 4,
                                             denom_mode=1)
-        assert np.all(O1 == 0.5), (S, order)
+        assert np.abs(O1 - 0.5).max() <= 4 * 2.0 ** -25, (S, order)
         O0, _, _ = oracle_mod.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, W.scale, S, order, 128, 4)
         if S == 1.0 and order == 0:
             # collapsed mass stays in l, so O comes out low on average (single rows
