@@ -53,12 +53,28 @@ def e4m3_cast(x, S: float = 1.0):
     return out
 
 
+def _launch(q, k, v, o, ctr, rows, *, causal, scale, S, kv_order, n_sink, block_n,
+            denominator, o_code, stream):
+    B, H, N, d = q.shape
+    fp8_attn_fwd_ex(q, k, v, o, B=B, H=H, H_kv=k.shape[1], N=N, d=d, causal=causal,
+                    scale=scale, S=S, kv_order=kv_order, n_sink=n_sink, o_dtype=o_code,
+                    block_n=block_n, denominator=denominator,
+                    collapse_ctr=None if ctr is None else ctr[0:1],
+                    collapse_sink_ctr=None if ctr is None else ctr[1:2],
+                    collapse_rows=rows, stream=stream)
+
+
 def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: float = 256.0,
               kv_order: int = KV_REVERSE, n_sink: int = 0, block_n: int = 0,
               denominator: int = DENOM_FP32_P,
               out_dtype=None, count_collapse: bool = False, per_row: bool = False,
-              out=None, stream=None):
-    """FP8 attention forward.  Returns (O, AttentionStats)."""
+              out=None, stream=None, host_chunks: int = 4):
+    """FP8 attention forward.  Returns (O, AttentionStats).
+
+    Host (CPU) tensors: the work is cut into up to ``host_chunks`` pieces along
+    the (batch, kv-head) axis; the copy of piece g+1 to the device runs on its
+    own stream while piece g computes, and piece g's output returns on a third
+    stream.  Pinned host memory makes those copies asynchronous."""
     import torch
     q, k, v = _as_bytes(q), _as_bytes(k), _as_bytes(v)
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
@@ -69,33 +85,77 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
         raise ValueError("k and v must be [B, H_kv, N, d] matching q")
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     o_code = {torch.bfloat16: O_BF16, torch.float32: O_F32}[out_dtype]
-    host = not q.is_cuda
-    dev = torch.device("cuda", torch.cuda.current_device()) if host else q.device
-    if host:
-        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    scale = scale if scale is not None else 1.0 / math.sqrt(d)
+    kw = dict(causal=causal, scale=scale, S=S, kv_order=kv_order, n_sink=n_sink,
+              block_n=block_n, denominator=denominator, o_code=o_code)
+    stats = AttentionStats()
+    if q.is_cuda:
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        dev = q.device
+        o = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype, device=dev)
+        ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
+        rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
+                if (count_collapse and per_row) else None)
+        _launch(q, k, v, o, ctr, rows, stream=stream, **kw)
+        if ctr is not None:
+            c = ctr.cpu()
+            stats.collapse, stats.collapse_sink_block = int(c[0]), int(c[1])
+            stats.collapse_rows = rows
+        return o, stats
+
+    # ---- host tensors: pipelined copies in, compute, copies out ----
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-    o = out if (out is not None and not host) else torch.empty((B, H, N, d), dtype=out_dtype,
-                                                               device=dev)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    group = H // H_kv
+    units = [(b, g) for b in range(B) for g in range(H_kv)]       # (batch, kv head)
+    nchunk = max(1, min(int(host_chunks), len(units)))
+    bounds = [len(units) * i // nchunk for i in range(nchunk + 1)]
+    res = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype,
+                                                  pin_memory=True)
+    compute = torch.cuda.current_stream(dev) if stream is None else stream
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
     rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
             if (count_collapse and per_row) else None)
-    fp8_attn_fwd_ex(q, k, v, o, B=B, H=H, H_kv=H_kv, N=N, d=d, causal=causal,
-                    scale=scale if scale is not None else 1.0 / math.sqrt(d), S=S,
-                    kv_order=kv_order, n_sink=n_sink, o_dtype=o_code, block_n=block_n,
-                    denominator=denominator,
-                    collapse_ctr=None if ctr is None else ctr[0:1],
-                    collapse_sink_ctr=None if ctr is None else ctr[1:2],
-                    collapse_rows=rows, stream=stream)
-    stats = AttentionStats()
-    if host:
-        res = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype,
-                                                      pin_memory=True)
-        res.copy_(o, non_blocking=True)
-        o = res
+    keep = []
+    for c in range(nchunk):
+        u0, u1 = bounds[c], bounds[c + 1]
+        # chunks never cross a batch element, so each is one contiguous slice
+        pieces = []
+        u = u0
+        while u < u1:
+            b = units[u][0]
+            e = u
+            while e < u1 and units[e][0] == b:
+                e += 1
+            pieces.append((b, units[u][1], units[e - 1][1] + 1))
+            u = e
+        for b, g0, g1 in pieces:
+            with torch.cuda.stream(s_in):
+                qd = q[b:b + 1, g0 * group:g1 * group].to(dev, non_blocking=True)
+                kd = k[b:b + 1, g0:g1].to(dev, non_blocking=True)
+                vd = v[b:b + 1, g0:g1].to(dev, non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            compute.wait_event(ev_in)
+            with torch.cuda.stream(compute):
+                od = torch.empty((1, (g1 - g0) * group, N, d), dtype=out_dtype, device=dev)
+                rd = None if rows is None else rows[b:b + 1, g0 * group:g1 * group]
+                _launch(qd, kd, vd, od, ctr, rd, stream=compute, **kw)
+                ev_c = torch.cuda.Event()
+                ev_c.record(compute)
+            s_out.wait_event(ev_c)
+            with torch.cuda.stream(s_out):
+                res[b:b + 1, g0 * group:g1 * group].copy_(od, non_blocking=True)
+            # the device buffers stay referenced until the output copy has run
+            for t in (qd, kd, vd, od):
+                t.record_stream(s_out)
+                t.record_stream(compute)
+            keep.append((qd, kd, vd, od))
+    s_out.synchronize()
+    compute.wait_stream(s_out)
     if ctr is not None:
         c = ctr.cpu()
         stats.collapse, stats.collapse_sink_block = int(c[0]), int(c[1])
         stats.collapse_rows = rows
-    elif host:
-        torch.cuda.current_stream().synchronize()
-    return o, stats
+    return res, stats
