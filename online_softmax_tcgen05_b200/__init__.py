@@ -68,7 +68,7 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
               kv_order: int = KV_REVERSE, n_sink: int = 0, block_n: int = 0,
               denominator: int = DENOM_FP32_P,
               out_dtype=None, count_collapse: bool = False, per_row: bool = False,
-              out=None, stream=None, host_chunks: int = 4):
+              out=None, stream=None, host_chunks: int = 8):
     """FP8 attention forward.  Returns (O, AttentionStats).
 
     Host (CPU) tensors: the work is cut into up to ``host_chunks`` pieces along
