@@ -36,6 +36,12 @@ CFG = dict(B=1, H=32, H_kv=8, N=32768, d=128, causal=1, S=256.0, kv_order=1, n_s
            delta=8.0, block_n=128)
 WORKLOAD = ("causal GQA prefill B=1 H=32/H_kv=8 N=32768 d=128 E4M3, sink construction "
             "n_sink=4 Delta=8, S=256, reverse KV order, O bf16, collapse counter on")
+# --shard heads: the long-context problem split by kv heads over the ranks
+CFG_LONG = dict(B=1, H=32, H_kv=8, N=131072, d=128, causal=1, S=256.0, kv_order=1, n_sink=4,
+                delta=10.0, block_n=128)
+WORKLOAD_LONG = ("long-context causal GQA B=1 H=32/H_kv=8 N=131072 d=128 E4M3, sink "
+                 "construction n_sink=4 Delta=10, S=256, reverse KV order, O bf16, collapse "
+                 "counter on; kv heads split over the ranks")
 METRIC = "FP8 attn fwd TFLOPS & % of B200 FP8 peak; P-collapse rate vs F(Δ,S)"
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -180,14 +186,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def make_inputs(seed, dev):
+def make_inputs(seed, dev, cfg=CFG, kv_heads=None):
     import torch
     import workload
     from online_softmax_tcgen05_b200 import e4m3_cast
-    W = workload.make_sink_workload(CFG["B"], CFG["H"], CFG["H_kv"], CFG["N"], CFG["d"],
-                                    CFG["n_sink"], CFG["delta"], seed=seed)
+    W = workload.make_sink_workload(cfg["B"], cfg["H"], cfg["H_kv"], cfg["N"], cfg["d"],
+                                    cfg["n_sink"], cfg["delta"], seed=seed, kv_heads=kv_heads)
     qkv = [e4m3_cast(torch.from_numpy(x).to(dev)) for x in (W.q, W.k, W.v)]
     return W, qkv
+
+
+def head_shard(rank, world, Hkv):
+    """kv heads [g0, g1) of this rank when a problem is split by kv heads."""
+    if Hkv % world:
+        raise ValueError("H_kv = %d does not split over %d ranks" % (Hkv, world))
+    per = Hkv // world
+    return rank * per, (rank + 1) * per
 
 
 def run_ours(args, rank, world, local_rank):
@@ -198,8 +212,14 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     fa.load_library()
     import workload
-    W, (q, k, v) = make_inputs(rank_seed(rank), dev)
-    B, H, Hkv, N, d = CFG["B"], CFG["H"], CFG["H_kv"], CFG["N"], CFG["d"]
+    strong = args.shard == "heads"
+    cfg = CFG_LONG if strong else CFG
+    if strong:
+        g0, g1 = head_shard(rank, world, cfg["H_kv"])
+        W, (q, k, v) = make_inputs(workload.CONFIG_SEED_BASE + 5, dev, cfg, kv_heads=(g0, g1))
+    else:
+        W, (q, k, v) = make_inputs(rank_seed(rank), dev)
+    B, H, Hkv, N, d = W.B, W.H, W.Hkv, W.N, W.d
     scale = 1.0 / math.sqrt(d)
     O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     ctr = torch.zeros(2, dtype=torch.int64, device=dev)
@@ -207,8 +227,8 @@ def run_ours(args, rank, world, local_rank):
 
     def step(count=True):
         fa.fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=Hkv, N=N, d=d, causal=True, scale=scale,
-                           S=CFG["S"], kv_order=CFG["kv_order"], n_sink=CFG["n_sink"],
-                           o_dtype=fa.O_BF16, block_n=CFG["block_n"],
+                           S=cfg["S"], kv_order=cfg["kv_order"], n_sink=cfg["n_sink"],
+                           o_dtype=fa.O_BF16, block_n=cfg["block_n"],
                            collapse_ctr=ctr[0:1] if count else None,
                            collapse_sink_ctr=ctr[1:2] if count else None, stream=stream)
 
@@ -238,8 +258,9 @@ def run_ours(args, rank, world, local_rank):
     collapse_total, collapse_sink = (int(x) for x in ctr.cpu().tolist())
     ms_off = timed(lambda: step(False), args.steps)
 
-    flops = algorithmic_flops(B, H, N, d, True)
+    flops = algorithmic_flops(B, H, N, d, True)          # this rank's work
     step_ms = ms_on / args.steps
+    # weak: every rank runs a whole problem; strong: the ranks share one problem
     value = job_tflops(flops, world, step_ms)
     kernel_tflops = flops / (step_ms * 1e-3) / 1e12
     peak, peak_src = peak_tflops()
@@ -258,8 +279,8 @@ def run_ours(args, rank, world, local_rank):
     oh = torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
 
     def e2e_step():
-        fa.attention(qh, kh, vh, causal=True, scale=scale, S=CFG["S"], kv_order=CFG["kv_order"],
-                     n_sink=CFG["n_sink"], block_n=CFG["block_n"], count_collapse=True, out=oh)
+        fa.attention(qh, kh, vh, causal=True, scale=scale, S=cfg["S"], kv_order=cfg["kv_order"],
+                     n_sink=cfg["n_sink"], block_n=cfg["block_n"], count_collapse=True, out=oh)
 
     for _ in range(max(1, args.warmup // 2)):
         e2e_step()
@@ -274,15 +295,18 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
     import oracle
-    pairs = world * B * H * (N - CFG["n_sink"]) * (N - CFG["n_sink"] + 1) // 2
+    pairs = world * B * H * (N - cfg["n_sink"]) * (N - cfg["n_sink"] + 1) // 2
     frac = collapse_total / args.steps / pairs
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD, **CFG, "per_rank": "independent prefill per GPU",
-                   "l2": "inputs 201 MB > 126 MB L2, no flush"},
+        "higher_is_better": True, "scaling": "strong" if strong else "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": ({"workload": WORKLOAD_LONG, **cfg, "per_rank": "kv heads split over the "
+                    "ranks; collapse counts all-reduced", "l2": "inputs 805 MB > 126 MB L2"}
+                   if strong else
+                   {"workload": WORKLOAD, **CFG, "per_rank": "independent prefill per GPU",
+                    "l2": "inputs 201 MB > 126 MB L2, no flush"}),
         "value_counter_off": round(job_tflops(flops, world, ms_off / args.steps), 2),
         "pct_of_fp8_peak": {"measured": round(kernel_tflops / peak, 4),
                             "nominal_4500": round(kernel_tflops / 4500.0, 4)},
@@ -293,49 +317,49 @@ def run_ours(args, rank, world, local_rank):
                      else peak_src},
         "collapse": {"fraction": frac, "count_per_step": collapse_total // args.steps // world,
                      "in_sink_block": collapse_sink // args.steps // world,
-                     "closed_form_forward_F": oracle.underflow_fraction_closed(CFG["delta"],
-                                                                               CFG["S"])},
+                     "closed_form_forward_F": oracle.underflow_fraction_closed(cfg["delta"],
+                                                                               cfg["S"])},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / e2e_steps, 3)},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(W, seconds_hint=True)
+        line["cpu_baseline"] = cpu_baseline(W, cfg, n_rows=8192 if strong else 32768)
     return line
 
 
-def sample_rows(n_rows, seed=7):
+def sample_rows(n_rows, seed=7, cfg=CFG):
     import numpy as np
     rng = np.random.default_rng(seed)
-    total = CFG["B"] * CFG["H"] * CFG["N"]
+    total = cfg["B"] * cfg["H"] * cfg["N"]
     return np.sort(rng.choice(total, n_rows, replace=False)).astype(np.int64)
 
 
-def oracle_sample(W, rows, Q8=None, K8=None, V8=None):
+def oracle_sample(W, rows, Q8=None, K8=None, V8=None, cfg=CFG):
     """Time the oracle's FP8 emulation on the given rows of the workload;
     returns (seconds, algorithmic FLOPs of those rows)."""
     import oracle
-    N, d = CFG["N"], CFG["d"]
+    N, d = W.N, W.d
     if Q8 is None:
         Q8, K8, V8 = (oracle.e4m3_encode(x) for x in (W.q, W.k, W.v))
     t0 = time.perf_counter()
-    oracle.attn_emulate(Q8, K8, V8, CFG["B"], CFG["H"], CFG["H_kv"], N, d, 1,
-                        1.0 / math.sqrt(d), CFG["S"], CFG["kv_order"], CFG["block_n"],
-                        CFG["n_sink"], o_bf16=True, rows=rows)
+    oracle.attn_emulate(Q8, K8, V8, W.B, W.H, W.Hkv, N, d, 1,
+                        1.0 / math.sqrt(d), cfg["S"], cfg["kv_order"], cfg["block_n"],
+                        cfg["n_sink"], o_bf16=True, rows=rows)
     dt = time.perf_counter() - t0
     flops = float(sum(4 * d * ((int(r) % N) + 1) for r in rows))
     return dt, flops, (Q8, K8, V8)
 
 
-def cpu_baseline(W, seconds_hint=True, n_rows=32768):
-    rows = sample_rows(n_rows)
-    dt, flops, _ = oracle_sample(W, rows)
+def cpu_baseline(W, cfg=CFG, n_rows=32768):
+    total = W.B * W.H * W.N
+    rows = sample_rows(n_rows, cfg=dict(cfg, H=W.H))
+    dt, flops, _ = oracle_sample(W, rows, cfg=cfg)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
             "kind": "oracle",
             "sample": "%d seeded random query rows of the %d (all heads and positions), "
-                      "FP8 pipeline emulation, %.1f s" % (n_rows, CFG["B"] * CFG["H"] * CFG["N"],
-                                                          dt)}
+                      "FP8 pipeline emulation, %.1f s" % (n_rows, total, dt)}
 
 
 def run_reference(args, rank, world):
@@ -378,6 +402,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["replica", "heads"], default="replica",
+                    help="replica: one independent prefill per rank (weak scaling); heads: "
+                         "the long-context problem split by kv heads (strong scaling)")
     ap.add_argument("--mode", choices=["full", "kernel"], default="full",
                     help="kernel: only the device-timed kernel loop (for profiling)")
     args = ap.parse_args()

@@ -116,39 +116,47 @@ def _unit_vectors(seed: int, B: int, Hkv: int, d: int) -> np.ndarray:
 
 
 def make_sink_workload(B: int, H: int, Hkv: int, N: int, d: int, n_sink: int = 4,
-                       delta: float = 8.0, seed: int = CONFIG_SEED_BASE) -> SinkWorkload:
+                       delta: float = 8.0, seed: int = CONFIG_SEED_BASE,
+                       kv_heads: tuple[int, int] | None = None) -> SinkWorkload:
     """Build Q, K, V (float32) with the sink construction described above.
 
     The draws do not depend on delta (common random numbers across a sweep):
     delta only sets the length of the u component of the sink keys.
-    """
+    kv_heads=(g0, g1) builds only kv heads g0..g1-1 and the query heads that
+    read them, with exactly the values the full problem has there (every
+    element's counter is its index in the full tensor)."""
     assert H % Hkv == 0 and 0 <= n_sink <= N
     group = H // Hkv
+    g0, g1 = (0, Hkv) if kv_heads is None else kv_heads
+    assert 0 <= g0 < g1 <= Hkv
+    nh, nq = g1 - g0, (g1 - g0) * group
     u = _unit_vectors(seed, B, Hkv, d)                        # [B,Hkv,d] f64
 
-    g = normals(seed, STREAM_Q, 0, B * H * N * d).reshape(B, H, N, d)
-    q = np.empty((B, H, N, d), dtype=np.float32)
+    q = np.empty((B, nq, N, d), dtype=np.float32)
     for b in range(B):
-        for h in range(H):
-            q[b, h] = g[b, h] + (8.0 * u[b, h // group]).astype(np.float32)
-    del g
+        g = normals(seed, STREAM_Q, (b * H + g0 * group) * N * d, nq * N * d).reshape(nq, N, d)
+        for j in range(nq):
+            q[b, j] = g[j] + (8.0 * u[b, g0 + j // group]).astype(np.float32)
+        del g
 
-    z = normals(seed, STREAM_K, 0, B * Hkv * N * d).reshape(B, Hkv, N, d)
-    k = np.empty((B, Hkv, N, d), dtype=np.float32)
+    k = np.empty((B, nh, N, d), dtype=np.float32)
     beta = delta * math.sqrt(d) / 8.0
     for b in range(B):
-        for h in range(Hkv):
-            uu = u[b, h]
-            zz = z[b, h].astype(np.float64)
+        z = normals(seed, STREAM_K, (b * Hkv + g0) * N * d, nh * N * d).reshape(nh, N, d)
+        for j in range(nh):
+            uu = u[b, g0 + j]
+            zz = z[j].astype(np.float64)
             proj = zz @ uu
             kk = zz - proj[:, None] * uu[None, :]
             if n_sink:
                 kk[:n_sink] = zz[:n_sink] + beta * uu[None, :]
-            k[b, h] = kk.astype(np.float32)
-    del z
+            k[b, j] = kk.astype(np.float32)
+        del z
 
-    v = normals(seed, STREAM_V, 0, B * Hkv * N * d).reshape(B, Hkv, N, d)
-    return SinkWorkload(q=q, k=k, v=v, B=B, H=H, Hkv=Hkv, N=N, d=d, n_sink=n_sink,
+    v = np.empty((B, nh, N, d), dtype=np.float32)
+    for b in range(B):
+        v[b] = normals(seed, STREAM_V, (b * Hkv + g0) * N * d, nh * N * d).reshape(nh, N, d)
+    return SinkWorkload(q=q, k=k, v=v, B=B, H=nq, Hkv=nh, N=N, d=d, n_sink=n_sink,
                         delta=float(delta), seed=seed)
 
 
