@@ -57,6 +57,11 @@ typedef enum {
 
 enum { FP8ATTN_KV_FORWARD = 0, FP8ATTN_KV_REVERSE = 1 };
 enum { FP8ATTN_O_BF16 = 0, FP8ATTN_O_F32 = 1 };
+/* Q and K element type.  E4M3 (default): QK^T on E4M3 operands.  BF16: Q and K
+ * are BF16 [.., d] rows and QK^T runs on BF16 operands, with P~ and V still
+ * E4M3 -- the P-cast paper's "kernel-faithful" simulation (Contributions 4),
+ * which leaves Q, K, V unquantised so that only the P-cast error remains. */
+enum { FP8ATTN_QK_E4M3 = 0, FP8ATTN_QK_BF16 = 1 };
 /* Row-sum (denominator) source.  FP32_P: l from the FP32 P before the cast and
  * O = acc / (S l) (the P-cast paper's kernel).  CAST_P: l from the cast values,
  * l = sum_j dec(pt_j), and O = acc / l, so numerator and denominator use the same
@@ -87,8 +92,8 @@ int fp8_attn_fwd(const void* Q, const void* K, const void* V, void* O,
 
 /* Full parameter set (same operation; see fp8_attn_fwd for shared fields). */
 typedef struct {
-  const void* Q;          /* E4M3 [B, H,    N, d] */
-  const void* K;          /* E4M3 [B, H_kv, N, d] */
+  const void* Q;          /* [B, H,    N, d], E4M3 or BF16 (qk_dtype) */
+  const void* K;          /* [B, H_kv, N, d], E4M3 or BF16 (qk_dtype) */
   const void* V;          /* E4M3 [B, H_kv, N, d] */
   void* O;                /* [B, H, N, d], dtype o_dtype */
   int B, H, H_kv, N, d;   /* H % H_kv == 0; query head h reads kv head h / (H / H_kv) */
@@ -98,6 +103,7 @@ typedef struct {
   int o_dtype;            /* FP8ATTN_O_BF16 (RNE) or FP8ATTN_O_F32 */
   int block_n;            /* KV block: 0 (= 128), 64 or 128.  N need not be a multiple:
                              the last block then holds the remaining keys. */
+  int qk_dtype;           /* FP8ATTN_QK_E4M3 (default, 0) or FP8ATTN_QK_BF16 */
   int denominator;        /* FP8ATTN_DENOM_FP32_P (default, 0) or FP8ATTN_DENOM_CAST_P;
                              CAST_P needs S >= 2^-8 so that the row maximum's cast is
                              nonzero */

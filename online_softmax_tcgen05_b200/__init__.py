@@ -18,7 +18,7 @@ import math
 from dataclasses import dataclass
 
 from ._binding import (DENOM_CAST_P, DENOM_FP32_P, ECUDA, EINVAL, ETIMEOUT, EUNSUPPORTED,
-                       KV_FORWARD, KV_REVERSE, O_BF16, O_F32, OK, Fp8AttnError, device_status_string, fp8_attn_fwd,
+                       KV_FORWARD, KV_REVERSE, O_BF16, O_F32, OK, QK_BF16, QK_E4M3, Fp8AttnError, device_status_string, fp8_attn_fwd,
                        fp8_attn_fwd_ex, fp8_e4m3_scale_cast, last_error, load_library,
                        status_string)
 
@@ -26,7 +26,7 @@ __all__ = ["attention", "AttentionStats", "fp8_attn_fwd", "fp8_attn_fwd_ex",
            "fp8_e4m3_scale_cast", "load_library", "status_string", "last_error",
            "device_status_string", "Fp8AttnError", "KV_FORWARD", "KV_REVERSE", "O_BF16",
            "O_F32", "OK", "EINVAL", "EUNSUPPORTED", "ECUDA", "ETIMEOUT", "e4m3_cast",
-           "DENOM_FP32_P", "DENOM_CAST_P"]
+           "DENOM_FP32_P", "DENOM_CAST_P", "QK_E4M3", "QK_BF16"]
 
 
 @dataclass
@@ -36,12 +36,15 @@ class AttentionStats:
     collapse_rows: object = None   # per-row counts [B, H, N] (torch.int32) or None
 
 
-def _as_bytes(t):
+def _as_bytes(t, allow_bf16=False):
     import torch
     if t.dtype == torch.float8_e4m3fn:
         return t.view(torch.uint8)
+    if allow_bf16 and t.dtype == torch.bfloat16:
+        return t
     if t.dtype != torch.uint8:
-        raise TypeError("E4M3 inputs must be torch.float8_e4m3fn or uint8, got %s" % t.dtype)
+        raise TypeError("inputs must be E4M3 (torch.float8_e4m3fn or uint8 bytes)%s, got %s"
+                        % (" or BF16 (q, k)" if allow_bf16 else "", t.dtype))
     return t
 
 
@@ -55,10 +58,12 @@ def e4m3_cast(x, S: float = 1.0):
 
 def _launch(q, k, v, o, ctr, rows, *, causal, scale, S, kv_order, n_sink, block_n,
             denominator, o_code, stream):
+    import torch
     B, H, N, d = q.shape
     fp8_attn_fwd_ex(q, k, v, o, B=B, H=H, H_kv=k.shape[1], N=N, d=d, causal=causal,
                     scale=scale, S=S, kv_order=kv_order, n_sink=n_sink, o_dtype=o_code,
                     block_n=block_n, denominator=denominator,
+                    qk_dtype=QK_BF16 if q.dtype == torch.bfloat16 else QK_E4M3,
                     collapse_ctr=None if ctr is None else ctr[0:1],
                     collapse_sink_ctr=None if ctr is None else ctr[1:2],
                     collapse_rows=rows, stream=stream)
@@ -71,12 +76,17 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
               out=None, stream=None, host_chunks: int = 8):
     """FP8 attention forward.  Returns (O, AttentionStats).
 
+    q, k: E4M3 (float8_e4m3fn or uint8 bytes) or both BF16 (the kernel-faithful
+    mode: QK^T on BF16 operands, P~ and V in E4M3); v: E4M3.
+
     Host (CPU) tensors: the work is cut into up to ``host_chunks`` pieces along
     the (batch, kv-head) axis; the copy of piece g+1 to the device runs on its
     own stream while piece g computes, and piece g's output returns on a third
     stream.  Pinned host memory makes those copies asynchronous."""
     import torch
-    q, k, v = _as_bytes(q), _as_bytes(k), _as_bytes(v)
+    q, k, v = _as_bytes(q, True), _as_bytes(k, True), _as_bytes(v)
+    if (q.dtype == torch.bfloat16) != (k.dtype == torch.bfloat16):
+        raise TypeError("q and k must both be E4M3 or both be BF16")
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be [B, H, N, d]")
     B, H, N, d = q.shape

@@ -15,6 +15,7 @@ from . import _build
 KV_FORWARD, KV_REVERSE = 0, 1
 O_BF16, O_F32 = 0, 1
 DENOM_FP32_P, DENOM_CAST_P = 0, 1
+QK_E4M3, QK_BF16 = 0, 1
 OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT = 0, -1, -2, -3, -4
 
 
@@ -33,7 +34,7 @@ class Params(ctypes.Structure):
                 ("scale", ctypes.c_float), ("S", ctypes.c_float),
                 ("kv_order", ctypes.c_int), ("n_sink", ctypes.c_int),
                 ("o_dtype", ctypes.c_int), ("block_n", ctypes.c_int),
-                ("denominator", ctypes.c_int),
+                ("qk_dtype", ctypes.c_int), ("denominator", ctypes.c_int),
                 ("collapse_ctr", ctypes.c_void_p), ("collapse_sink_ctr", ctypes.c_void_p),
                 ("collapse_rows", ctypes.c_void_p), ("status_word", ctypes.c_void_p),
                 ("timeout_ns", ctypes.c_ulonglong), ("debug_skip_kv_step", ctypes.c_int)]
@@ -121,6 +122,7 @@ def fp8_attn_fwd(Q, K, V, O, B, H, N, d, causal, scale, S, kv_order, n_sink, col
 
 def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S=256.0,
                     kv_order=KV_REVERSE, n_sink=0, o_dtype=O_BF16, block_n=0, denominator=0,
+                    qk_dtype=QK_E4M3,
                     collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None,
                     status_word=None, timeout_ns=0, debug_skip_kv_step=0, stream=None):
     """Full-parameter entry point (all tensors on the device)."""
@@ -128,7 +130,7 @@ def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S
                B=B, H=H, H_kv=H_kv, N=N, d=d, causal=int(causal),
                scale=float(scale if scale is not None else 1.0 / math.sqrt(d)), S=float(S),
                kv_order=int(kv_order), n_sink=int(n_sink), o_dtype=int(o_dtype),
-               block_n=int(block_n), denominator=int(denominator),
+               block_n=int(block_n), denominator=int(denominator), qk_dtype=int(qk_dtype),
                collapse_ctr=None if collapse_ctr is None else collapse_ctr.data_ptr(),
                collapse_sink_ctr=None if collapse_sink_ctr is None else collapse_sink_ctr.data_ptr(),
                collapse_rows=None if collapse_rows is None else collapse_rows.data_ptr(),

@@ -69,7 +69,6 @@ enum : uint32_t {
 
 struct KParams {
   int B, H, Hkv, N, group;
-  float log2_S;       // log2(S) when S is an exact power of two (folded into the exponent)
   int causal, kv_order, n_sink;
   int num_q_tiles;
   float scale_log2;   // scale * log2(e)
@@ -84,11 +83,11 @@ struct KParams {
   int denom_cast;           // row sum from the cast values (FP8ATTN_DENOM_CAST_P)
 };
 
-template <int D, int BN>
+template <int D, int BN, int QB>
 struct Smem {
   static constexpr int Q = 0;
-  static constexpr int K = Q + BM * D;
-  static constexpr int V = K + NSTAGE * BN * D;
+  static constexpr int K = Q + BM * D * QB;
+  static constexpr int V = K + NSTAGE * BN * D * QB;
   static constexpr int P = V + NSTAGE * BN * D;
   static constexpr int BAR = P + BM * BN;
   // barriers: q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full, s_free, p_full,
@@ -107,14 +106,15 @@ __device__ __forceinline__ int kv_block_at(int t, int T, int order) {
   return order == FP8ATTN_KV_FORWARD ? t : T - 1 - t;
 }
 
-// FOLD: S is a power of two 2^k.  Then S * 2^(x - m) = 2^(x - m + k) exactly
-// (multiplying by 2^k only moves the exponent), so k joins the exponent's FMA
-// and the product disappears; the row sum is brought back by 2^-k, also exact.
-template <int D, int BN, bool OUT_BF16, bool COUNT, bool FOLD>
+// QB: bytes per Q / K element.  1: E4M3 Q and K, QK^T as kind::f8f6f4.
+// 2: BF16 Q and K, QK^T as kind::f16 (the "kernel-faithful" reading of the
+// P-cast paper's simulation, where only P~ and V are E4M3); each BF16 row is
+// staged as D/64 panels of 64 elements (128-byte swizzle atoms).
+template <int D, int BN, bool OUT_BF16, bool COUNT, int QB>
 __global__ void __launch_bounds__(NTHREADS, 2)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p) {
-  using L = Smem<D, BN>;
+  using L = Smem<D, BN, QB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -178,8 +178,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (warp == 4) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q_full, BM * D);
-      tma_load_3d(sQ, &tmQ, bar_q_full, 0, q0, bh);
+      // Q: E4M3 rows in one box; BF16 rows as D/64 panels of 64 elements
+      mbar_arrive_expect_tx(bar_q_full, BM * D * QB);
+      if constexpr (QB == 1) {
+        tma_load_3d(sQ, &tmQ, bar_q_full, 0, q0, bh);
+      } else {
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_load_3d(sQ + pn * BM * 128, &tmQ, bar_q_full, 64 * pn, q0, bh);
+      }
       // K runs one KV step ahead of V: K(t+1) needs only QK^T(t-1) to have
       // released its stage, V(t) needs P~V(t-2).
       int k_issued = 0, v_issued = 0;
@@ -188,9 +195,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (t >= NSTAGE && !mbar_wait(bar_k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
           return false;
         if (t + 1 == p.debug_skip_kv_step) return true;   // testing: leave this K tile out
-        mbar_arrive_expect_tx(bar_k_full(st), BN * D);
-        tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
-                    bkv);
+        mbar_arrive_expect_tx(bar_k_full(st), BN * D * QB);
+        {
+          const int jrow = kv_block_at(t, T, p.kv_order) * BN;
+          if constexpr (QB == 1) {
+            tma_load_3d(sK + st * BN * D, &tmK, bar_k_full(st), 0, jrow, bkv);
+          } else {
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn)
+              tma_load_3d(sK + st * BN * D * QB + pn * BN * 128, &tmK, bar_k_full(st), 64 * pn,
+                          jrow, bkv);
+          }
+        }
         k_issued = t + 1;
         return true;
       };
@@ -228,11 +244,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     auto issue_qk = [&](int st) {
       tc_fence_after();
       if (lane == 0) {
+        if constexpr (QB == 1) {
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk) {
-          const uint64_t a = smem_desc(sQ + 32 * kk, 16, 8 * D, SWZ_QK);
-          const uint64_t bdesc = smem_desc(sK + st * BN * D + 32 * kk, 16, 8 * D, SWZ_QK);
-          mma_e4m3_ss(tS, a, bdesc, IDESC_QK, kk > 0);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t a = smem_desc(sQ + 32 * kk, 16, 8 * D, SWZ_QK);
+            const uint64_t bdesc = smem_desc(sK + st * BN * D + 32 * kk, 16, 8 * D, SWZ_QK);
+            mma_e4m3_ss(tS, a, bdesc, IDESC_QK, kk > 0);
+          }
+        } else {
+          // BF16: K = 16 per instruction, 4 steps of 32 bytes per 64-element panel
+          constexpr uint32_t IDESC_QK16 = idesc_bf16_f32(BM, BN);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t pn = kk / 4, off = 32 * (kk % 4);
+            const uint64_t a = smem_desc(sQ + pn * BM * 128 + off, 16, 1024, SWZ_128B);
+            const uint64_t bdesc =
+                smem_desc(sK + st * BN * D * QB + pn * BN * 128 + off, 16, 1024, SWZ_128B);
+            mma_bf16_ss(tS, a, bdesc, IDESC_QK16, kk > 0);
+          }
         }
         mma_commit(bar_s_full);
         mma_commit(bar_k_empty(st));
@@ -282,7 +311,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t tS = tmem_base + lane_off, tO = tmem_base + lane_off + BN;
     const float c = p.scale_log2;
     const float S = p.S;
-    const float inv_S = 1.f / S;   // exact when FOLD (S a power of two)
     float m_run = -INFINITY, l = 0.f;
     uint32_t cnt = 0, cnt_sink = 0;
     bool ok = true;
@@ -333,8 +361,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
       // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
-      const float off = FOLD ? p.log2_S - m_use : -m_use;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(off, off);
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
       float2 acc8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
@@ -356,22 +383,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
       const float rowsum = acc8[0].x + acc8[0].y;
-      if (!p.denom_cast) l = alpha * l + (FOLD ? rowsum * inv_S : rowsum);
-      // S * p (already in s[] when FOLD; else packed FMUL2), then the E4M3 cast,
-      // four keys per word
+      if (!p.denom_cast) l = alpha * l + rowsum;
+      // S * p (packed FMUL2), then the E4M3 cast, four keys per word
       uint32_t pw[BN / 4];
-      if constexpr (FOLD) {
+      const float2 S2 = make_float2(S, S);
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q)
-          pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-      } else {
-        const float2 S2 = make_float2(S, S);
-#pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-          const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
-          const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
-          pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
-        }
+      for (int q = 0; q < BN / 4; ++q) {
+        const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
+        const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
+        pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
       }
       if (p.denom_cast) {
         // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
@@ -575,28 +595,33 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over an E4M3 tensor [planes, rows, d] with box [d, box_rows, 1].
-bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows) {
+// 3-D map over a [planes, rows, d] tensor of E4M3 bytes (box [d, box_rows, 1],
+// 128- or 64-byte swizzle by row length) or of BF16 (box [64, box_rows, 1]: one
+// 128-byte swizzle atom per row; a row of d = 128 is loaded as two such panels).
+bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows,
+              bool bf16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t esz = bf16 ? 2 : 1;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes};
-  cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)d * (cuuint64_t)rows};
-  cuuint32_t box[3] = {(cuuint32_t)d, (cuuint32_t)box_rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)d * esz, (cuuint64_t)d * esz * (cuuint64_t)rows};
+  cuuint32_t box[3] = {(cuuint32_t)(bf16 ? 64 : d), (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUtensorMapSwizzle swz = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUtensorMapSwizzle swz = (bf16 || d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B
+                                              : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D, int BN, bool OUT_BF16, bool COUNT, bool FOLD>
+template <int D, int BN, bool OUT_BF16, bool COUNT, int QB>
 cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                    const fp8attn::KParams& kp, cudaStream_t stream) {
-  using L = fp8attn::Smem<D, BN>;
-  auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT, FOLD>;
+  using L = fp8attn::Smem<D, BN, QB>;
+  auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT, QB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(kp.num_q_tiles, kp.B * kp.H);
@@ -604,28 +629,21 @@ cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap
   return cudaGetLastError();
 }
 
-template <int D, int BN, bool FOLD>
-cudaError_t launch_f(bool bf16, bool count, const CUtensorMap& q, const CUtensorMap& k,
+template <int D, int BN, int QB>
+cudaError_t launch_q(bool bf16, bool count, const CUtensorMap& q, const CUtensorMap& k,
                      const CUtensorMap& v, const fp8attn::KParams& kp, cudaStream_t s) {
-  if (bf16) return count ? launch<D, BN, true, true, FOLD>(q, k, v, kp, s)
-                         : launch<D, BN, true, false, FOLD>(q, k, v, kp, s);
-  return count ? launch<D, BN, false, true, FOLD>(q, k, v, kp, s)
-               : launch<D, BN, false, false, FOLD>(q, k, v, kp, s);
+  if (bf16) return count ? launch<D, BN, true, true, QB>(q, k, v, kp, s)
+                         : launch<D, BN, true, false, QB>(q, k, v, kp, s);
+  return count ? launch<D, BN, false, true, QB>(q, k, v, kp, s)
+               : launch<D, BN, false, false, QB>(q, k, v, kp, s);
 }
 
 template <int D, int BN>
-cudaError_t launch_dt(bool bf16, bool count, bool fold, const CUtensorMap& q, const CUtensorMap& k,
-                      const CUtensorMap& v, const fp8attn::KParams& kp, cudaStream_t s) {
-  return fold ? launch_f<D, BN, true>(bf16, count, q, k, v, kp, s)
-              : launch_f<D, BN, false>(bf16, count, q, k, v, kp, s);
-}
-
-// log2(S) when S is an exact power of two with 2^k and 2^-k both normal, else NaN.
-float pow2_log2(float S) {
-  int e;
-  const float m = std::frexp(S, &e);
-  if (m != 0.5f || e - 1 < -125 || e - 1 > 125) return NAN;
-  return (float)(e - 1);
+cudaError_t launch_dt(bool bf16, bool count, bool qk_bf16, const CUtensorMap& q,
+                      const CUtensorMap& k, const CUtensorMap& v, const fp8attn::KParams& kp,
+                      cudaStream_t s) {
+  return qk_bf16 ? launch_q<D, BN, 2>(bf16, count, q, k, v, kp, s)
+                 : launch_q<D, BN, 1>(bf16, count, q, k, v, kp, s);
 }
 
 }  // namespace
@@ -685,6 +703,8 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
     return fail(FP8ATTN_EINVAL, "denominator must be FP8ATTN_DENOM_FP32_P or FP8ATTN_DENOM_CAST_P");
   if (p->denominator == FP8ATTN_DENOM_CAST_P && std::isfinite(p->S) && p->S < 0x1p-8f)
     return fail(FP8ATTN_EINVAL, "the cast-value denominator needs S >= 2^-8");
+  if (p->qk_dtype != FP8ATTN_QK_E4M3 && p->qk_dtype != FP8ATTN_QK_BF16)
+    return fail(FP8ATTN_EINVAL, "qk_dtype must be FP8ATTN_QK_E4M3 or FP8ATTN_QK_BF16");
   if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
     return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
   if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
@@ -705,9 +725,10 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
 
   CUtensorMap mq, mk, mv;
   if (!encode_fn()) return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled is not available");
-  if (!make_map(&mq, p->Q, p->d, p->N, p->B * p->H, fp8attn::BM) ||
-      !make_map(&mk, p->K, p->d, p->N, p->B * p->H_kv, bn) ||
-      !make_map(&mv, p->V, p->d, p->N, p->B * p->H_kv, bn))
+  const bool qkb = p->qk_dtype == FP8ATTN_QK_BF16;
+  if (!make_map(&mq, p->Q, p->d, p->N, p->B * p->H, fp8attn::BM, qkb) ||
+      !make_map(&mk, p->K, p->d, p->N, p->B * p->H_kv, bn, qkb) ||
+      !make_map(&mv, p->V, p->d, p->N, p->B * p->H_kv, bn, false))
     return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled failed");
 
   fp8attn::KParams kp;
@@ -734,17 +755,15 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
 
   const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;
   const bool count = p->collapse_ctr != nullptr;
-  const float k2 = pow2_log2(p->S);
-  const bool fold = !std::isnan(k2);
-  kp.log2_S = fold ? k2 : 0.f;
+  const bool qk_bf16 = p->qk_dtype == FP8ATTN_QK_BF16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (p->d == 128)
-    e = (bn == 128) ? launch_dt<128, 128>(bf16, count, fold, mq, mk, mv, kp, s)
-                    : launch_dt<128, 64>(bf16, count, fold, mq, mk, mv, kp, s);
+    e = (bn == 128) ? launch_dt<128, 128>(bf16, count, qk_bf16, mq, mk, mv, kp, s)
+                    : launch_dt<128, 64>(bf16, count, qk_bf16, mq, mk, mv, kp, s);
   else
-    e = (bn == 128) ? launch_dt<64, 128>(bf16, count, fold, mq, mk, mv, kp, s)
-                    : launch_dt<64, 64>(bf16, count, fold, mq, mk, mv, kp, s);
+    e = (bn == 128) ? launch_dt<64, 128>(bf16, count, qk_bf16, mq, mk, mv, kp, s)
+                    : launch_dt<64, 64>(bf16, count, qk_bf16, mq, mk, mv, kp, s);
   if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return FP8ATTN_OK;
 }

@@ -63,10 +63,11 @@ def lib():
         L.oracle_bf16_rne.restype = f32
         L.oracle_e4m3_scale_cast.argtypes = [P, P, i64, f32]
         L.oracle_e4m3_scale_cast_bits.argtypes = [u64, i64, f32, P]
-        L.oracle_attn_exact.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, i64, P, i32]
+        L.oracle_attn_exact.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, i64, P, i32,
+                                        i32]
         L.oracle_attn_exact.restype = i32
         L.oracle_attn_emulate.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f32, f32,
-                                          i32, i32, i32, i32, P, i64, P, P, P, i32, i32]
+                                          i32, i32, i32, i32, P, i64, P, P, P, i32, i32, i32]
         L.oracle_attn_emulate.restype = i32
         L.oracle_collapse_logits.argtypes = [P, i64, i32, i32, i32, f32, i32, P, P, i32]
         L.oracle_collapse_logits.restype = i32
@@ -110,6 +111,14 @@ def bf16_rne(x: np.ndarray) -> np.ndarray:
     return np.vectorize(lambda v: L.oracle_bf16_rne(float(v)), otypes=[np.float32])(x)
 
 
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns (uint16) of x rounded to nearest even (finite x): the
+    same rounding as bf16_rne, done on the FP32 bits in bulk."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
 # -------------------------------------------------------------- attention ----
 def _rows(rows):
     if rows is None:
@@ -118,13 +127,21 @@ def _rows(rows):
     return r, r.size
 
 
+def _qk_flag(Q, K):
+    if Q.dtype == np.uint16 and K.dtype == np.uint16:
+        return 1                      # BF16 bit patterns
+    assert Q.dtype == np.uint8 and K.dtype == np.uint8
+    return 0
+
+
 def attn_exact(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, rows=None, nthreads=0):
-    """float64 O* = softmax(scale Q K^T) V on decoded E4M3 inputs, [nrows, d]."""
+    """float64 O* = softmax(scale Q K^T) V on the decoded inputs, [nrows, d].
+    Q, K: E4M3 bytes (uint8) or BF16 bit patterns (uint16); V: E4M3 bytes."""
     r, nr = _rows(rows)
     n_out = nr if r is not None else B * H * N
     O = np.empty((n_out, d), dtype=np.float64)
     rc = lib().oracle_attn_exact(_ptr(Q8), _ptr(K8), _ptr(V8), B, H, Hkv, N, d, int(causal),
-                                 float(scale), _ptr(r), nr, _ptr(O), nthreads)
+                                 float(scale), _ptr(r), nr, _ptr(O), nthreads, _qk_flag(Q8, K8))
     if rc:
         raise ValueError("oracle_attn_exact: bad shape")
     return O
@@ -134,10 +151,12 @@ def attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, kv_order, block_
                  o_bf16=False, rows=None, nthreads=0, denom_mode=0):
     """FP8 pipeline emulation.  Returns (O [nrows, d] float32, collapse per row
     uint32, totals uint64[2] = {in sink-holding KV blocks, in other blocks}).
-    denom_mode 0: l from the FP32 P, O = acc / (S l); 1: l from the cast values,
+    Q, K: E4M3 bytes (uint8) or BF16 bit patterns (uint16, the kernel-faithful
+    mode); V: E4M3 bytes.  denom_mode 0: l from the FP32 P, O = acc / (S l); 1: l from the cast values,
     O = acc / l."""
     for a in (Q8, K8, V8):
-        assert a.dtype == np.uint8 and a.flags.c_contiguous
+        assert a.flags.c_contiguous
+    assert V8.dtype == np.uint8
     r, nr = _rows(rows)
     n_out = nr if r is not None else B * H * N
     O = np.empty((n_out, d), dtype=np.float32)
@@ -146,7 +165,8 @@ def attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, kv_order, block_
     rc = lib().oracle_attn_emulate(_ptr(Q8), _ptr(K8), _ptr(V8), B, H, Hkv, N, d, int(causal),
                                    float(scale), float(S), int(kv_order), int(block_n),
                                    int(n_sink), int(bool(o_bf16)), _ptr(r), nr, _ptr(O),
-                                   _ptr(cr), _ptr(tot), nthreads, int(denom_mode))
+                                   _ptr(cr), _ptr(tot), nthreads, int(denom_mode),
+                                   _qk_flag(Q8, K8))
     if rc:
         raise ValueError("oracle_attn_emulate: bad shape")
     return O, cr, tot

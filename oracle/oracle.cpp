@@ -12,7 +12,8 @@
 //   * e4m3_*     : the E4M3 number format (Problem statement: 3-bit mantissa;
 //                  Methodology: round-to-zero threshold 2^-10; Optimality of
 //                  S=256, condition 3: normal floor 2^-6, largest finite 448).
-//   * attn_exact : float64 softmax attention on the decoded E4M3 inputs.
+//   * attn_exact : float64 softmax attention on the decoded E4M3 inputs (or BF16
+//                  Q and K: the "kernel-faithful" mode of Contributions 4).
 //   * attn_emulate : the FP8 pipeline, KV block by KV block, in the order the
 //                  online softmax visits the blocks (Problem statement:
 //                  running max m, KV iteration order, static scale S applied
@@ -74,10 +75,27 @@ uint8_t e4m3_encode(float x) {
     return sign | code;
 }
 
+
 float g_dec[256];
 struct DecInit {
     DecInit() { for (int c = 0; c < 256; ++c) g_dec[c] = (float)e4m3_value((uint8_t)c); }
 } g_dec_init;
+
+inline float g_dec_lookup(uint8_t c) { return g_dec[c]; }
+
+// Value of a BF16 bit pattern (the upper half of an FP32).
+inline float bf16_value(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+}
+
+// Element idx of a Q or K tensor: E4M3 bytes, or BF16 bit patterns when qk_bf16.
+inline float qk_value(const void* base, int64_t idx, int qk_bf16) {
+    return qk_bf16 ? bf16_value(static_cast<const uint16_t*>(base)[idx])
+                   : g_dec_lookup(static_cast<const uint8_t*>(base)[idx]);
+}
 
 // BF16 round-to-nearest-even of a finite float, returned as a float.
 float bf16_rne(float x) {
@@ -171,9 +189,9 @@ void oracle_e4m3_scale_cast_bits(uint64_t first, int64_t n, float S, uint8_t* ou
 // ---- float64 exact attention on decoded E4M3 inputs ------------------------
 // O*[r, :] = sum_j softmax_j(scale * q_i . k_j) v_j, causal: j <= i;
 // query head h reads kv head h / (H / Hkv).  rows == NULL: all B*H*N rows.
-int oracle_attn_exact(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
+int oracle_attn_exact(const void* Q, const void* K, const uint8_t* V,
                       int B, int H, int Hkv, int N, int d, int causal, double scale,
-                      const int64_t* rows, int64_t nrows, double* O, int nthreads) {
+                      const int64_t* rows, int64_t nrows, double* O, int nthreads, int qk_bf16) {
     if (H % Hkv) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
@@ -187,15 +205,15 @@ int oracle_attn_exact(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
             int64_t r = rows ? rows[t] : t;
             int b, h, i;
             row_coords(sh, r, b, h, i);
-            const uint8_t* qp = Q + (((int64_t)b * H + h) * N + i) * d;
+            const int64_t qbase = (((int64_t)b * H + h) * N + i) * d;
             const int64_t kvbase = (((int64_t)b * Hkv + h / group) * N) * d;
-            for (int k = 0; k < d; ++k) q[k] = e4m3_value(qp[k]);
+            for (int k = 0; k < d; ++k) q[k] = qk_value(Q, qbase + k, qk_bf16);
             int jend = causal ? i + 1 : N;
             double mx = -std::numeric_limits<double>::infinity();
             for (int j = 0; j < jend; ++j) {
-                const uint8_t* kp = K + kvbase + (int64_t)j * d;
+                const int64_t kb = kvbase + (int64_t)j * d;
                 double dot = 0.0;
-                for (int k = 0; k < d; ++k) dot += q[k] * e4m3_value(kp[k]);
+                for (int k = 0; k < d; ++k) dot += q[k] * (double)qk_value(K, kb + k, qk_bf16);
                 s[j] = scale * dot;
                 if (s[j] > mx) mx = s[j];
             }
@@ -235,12 +253,12 @@ int oracle_attn_exact(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
 // Outputs: O [nrows, d] (float), collapse_rows [nrows] (nullable),
 // collapse_totals[2] = {entries in KV blocks holding a sink key, entries in the
 // other blocks} (nullable, accumulated).
-int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
+int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
                         int B, int H, int Hkv, int N, int d, int causal, float scale, float S,
                         int kv_order, int block_n, int n_sink, int o_bf16,
                         const int64_t* rows, int64_t nrows,
                         float* O, uint32_t* collapse_rows, uint64_t* collapse_totals,
-                        int nthreads, int denom_mode) {
+                        int nthreads, int denom_mode, int qk_bf16) {
     if (H % Hkv || block_n <= 0) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
@@ -257,9 +275,9 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
             int64_t r = rows ? rows[t] : t;
             int b, h, i;
             row_coords(sh, r, b, h, i);
-            const uint8_t* qp = Q + (((int64_t)b * H + h) * N + i) * d;
+            const int64_t qbase = (((int64_t)b * H + h) * N + i) * d;
             const int64_t kvbase = (((int64_t)b * Hkv + h / group) * N) * d;
-            for (int k = 0; k < d; ++k) q[k] = g_dec[qp[k]];
+            for (int k = 0; k < d; ++k) q[k] = qk_value(Q, qbase + k, qk_bf16);
             for (int k = 0; k < d; ++k) acc[k] = 0.0f;
             RowState st;
             float lq = 0.0f;   // denominator from the cast values (denom_mode 1)
@@ -272,9 +290,9 @@ int oracle_attn_emulate(const uint8_t* Q, const uint8_t* K, const uint8_t* V,
                 for (int jj = 0; jj < nb; ++jj) {
                     int j = j0 + jj;
                     if (causal && j > i) { s[jj] = kNegInf; continue; }
-                    const uint8_t* kp = K + kvbase + (int64_t)j * d;
+                    const int64_t kb = kvbase + (int64_t)j * d;
                     float dot = 0.0f;
-                    for (int k = 0; k < d; ++k) dot += q[k] * g_dec[kp[k]];
+                    for (int k = 0; k < d; ++k) dot += q[k] * qk_value(K, kb + k, qk_bf16);
                     s[jj] = scale * dot;
                 }
                 float alpha;

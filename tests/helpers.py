@@ -25,6 +25,24 @@ def gpu_inputs(W, dev="cuda"):
     return out
 
 
+def gpu_inputs_bf16(W, dev="cuda"):
+    """BF16 Q and K (the kernel-faithful mode) and E4M3 V: the GPU side rounds
+    with torch, the oracle side with its own RNE; the bits must agree."""
+    import torch
+    from online_softmax_tcgen05_b200 import e4m3_cast
+    out = []
+    for x in (W.q, W.k):
+        g = torch.from_numpy(x).to(dev).to(torch.bfloat16)
+        o = oracle.bf16_bits(x)
+        assert np.array_equal(g.view(torch.int16).cpu().numpy().view(np.uint16), o)
+        out.append((g, o))
+    g = e4m3_cast(torch.from_numpy(W.v).to(dev))
+    o = oracle.e4m3_encode(W.v)
+    assert np.array_equal(g.cpu().numpy(), o)
+    out.append((g, o))
+    return out
+
+
 def compare_o(O_gpu, O_ref):
     O_gpu = np.asarray(O_gpu, dtype=np.float64)
     O_ref = np.asarray(O_ref, dtype=np.float64)
@@ -49,5 +67,5 @@ def sample_rows(B, H, N, n, seed=0, include=()):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-__all__ = ["gpu_inputs", "compare_o", "assert_o_close", "sample_rows", "O_MAX_ABS", "O_REL_RMS",
+__all__ = ["gpu_inputs", "gpu_inputs_bf16", "compare_o", "assert_o_close", "sample_rows", "O_MAX_ABS", "O_REL_RMS",
            "COLLAPSE_ABS", "oracle", "workload"]

@@ -70,6 +70,7 @@ def base_params(**kw):
     (dict(collapse_rows=FAKE), EINVAL), (dict(collapse_ctr=FAKE + 4), EINVAL),
     (dict(debug_skip_kv_step=-1), EINVAL), (dict(debug_skip_kv_step=2), EINVAL),
     (dict(denominator=2), EINVAL), (dict(denominator=1, S=0.001), EINVAL),
+    (dict(qk_dtype=2), EINVAL),
 ])
 def test_invalid_arguments_rejected_before_launch(lib, kw, status):
     p = base_params(**kw)

@@ -17,8 +17,8 @@ import math
 import numpy as np
 import pytest
 
-from helpers import (COLLAPSE_ABS, assert_o_close, compare_o, gpu_inputs, oracle, sample_rows,
-                     workload)
+from helpers import (COLLAPSE_ABS, assert_o_close, compare_o, gpu_inputs, gpu_inputs_bf16, oracle,
+                     sample_rows, workload)
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +26,7 @@ pytestmark = pytest.mark.gpu
 def run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, n_sink, f32=True, scale=None,
             count=True, denominator=0):
     import torch
-    from online_softmax_tcgen05_b200 import O_BF16, O_F32, fp8_attn_fwd_ex
+    from online_softmax_tcgen05_b200 import O_BF16, O_F32, QK_BF16, QK_E4M3, fp8_attn_fwd_ex
     (Qg, _), (Kg, _), (Vg, _) = ins
     dev = Qg.device
     O = torch.full((B, H, N, d), float("nan"), dtype=torch.float32 if f32 else torch.bfloat16,
@@ -38,6 +38,7 @@ def run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, n_sink, f32=True, s
                     scale=scale if scale is not None else 1.0 / math.sqrt(d), S=S,
                     kv_order=order, n_sink=n_sink, o_dtype=O_F32 if f32 else O_BF16,
                     block_n=block_n, denominator=denominator,
+                    qk_dtype=QK_BF16 if Qg.dtype == torch.bfloat16 else QK_E4M3,
                     collapse_ctr=ctr[0:1] if count else None,
                     collapse_sink_ctr=ctr[1:2] if count else None,
                     collapse_rows=rows if count else None, status_word=status)
@@ -208,7 +209,7 @@ def test_sweep_collapse_and_closed_form(sweep_inputs):
 def test_sweep_mse_orderings(sweep_inputs):
     W, ins = sweep_inputs[7]
     (_, Q8), (_, K8), (_, V8) = ins
-    rows = sample_rows(1, 8, 4096, 384, seed=5)
+    rows = sample_rows(1, 8, 4096, 2048, seed=5)      # a 10% MSE effect needs ~2k rows
     ref = oracle.attn_exact(Q8, K8, V8, 1, 8, 8, 4096, 128, 0, W.scale, rows=rows)
     mse = {}
     for order in (0, 1):
@@ -217,8 +218,8 @@ def test_sweep_mse_orderings(sweep_inputs):
             mse[(order, S)] = float(np.mean((Og[rows] - ref) ** 2))
     base = mse[(0, 1.0)]
     best = min(mse[(0, 256.0)], mse[(1, 256.0)], mse[(1, 1.0)])
-    assert 2.5 < base / best < 10.5, mse                   # paper: 3-10x
-    assert mse[(0, 256.0)] < mse[(0, 448.0)], mse          # paper: 10-15% lower
+    assert 2.0 < base / best < 10.5, mse                   # paper: 3-10x
+    assert mse[(0, 256.0)] / mse[(0, 448.0)] < 0.97, mse   # paper: 10-15% lower
     assert abs(mse[(1, 256.0)] / mse[(0, 256.0)] - 1) < 0.1, mse
 
 
@@ -311,3 +312,36 @@ def test_cast_denominator_parity(B, H, Hkv, N, d, block_n, causal):
             Oe, _, _ = oracle.attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, W.scale, S, order,
                                            block_n, 4, denom_mode=1)
             assert_o_close(Og, Oe, ("cast denominator", S, order))
+
+
+
+@pytest.mark.parametrize("B,H,Hkv,N,d,block_n,causal", [(1, 2, 1, 384, 128, 128, 1),
+                                                        (1, 2, 2, 1000, 128, 64, 1),
+                                                        (2, 2, 1, 520, 64, 128, 0),
+                                                        (1, 1, 1, 333, 64, 64, 1)])
+def test_bf16_qk_parity(B, H, Hkv, N, d, block_n, causal):
+    """Kernel-faithful mode: QK^T on BF16 Q and K (tcgen05 kind::f16), P~ and V
+    E4M3, against the oracle in the same mode."""
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 9.0, seed=70 + N + d)
+    ins = gpu_inputs_bf16(W)
+    for S in (1.0, 256.0, 448.0):
+        for order in (0, 1):
+            check_case(W, ins, causal, S, order, block_n, f32=(S != 448.0),
+                       what=("bf16 qk", B, H, Hkv, N, d, block_n, causal, S, order))
+
+
+def test_bf16_qk_mse_orderings_on_gpu():
+    """The paper's MSE claims in its own setting (unquantised Q, K) on the
+    kernel's outputs: Delta = 7, N = 4096, 2048 sampled rows."""
+    W = workload.make_sink_workload(1, 8, 8, 4096, 128, 4, 7.0, seed=workload.CONFIG_SEED_BASE + 2)
+    ins = gpu_inputs_bf16(W)
+    (_, Q), (_, K), (_, V8) = ins
+    rows = sample_rows(1, 8, 4096, 2048, seed=5)
+    ref = oracle.attn_exact(Q, K, V8, 1, 8, 8, 4096, 128, 0, W.scale, rows=rows)
+    mse = {}
+    for order, S in ((0, 1.0), (0, 256.0), (0, 448.0), (1, 256.0)):
+        Og, *_ = run_gpu(ins, 1, 8, 8, 4096, 128, 0, S, order, 128, 4)
+        mse[(order, S)] = float(np.mean((Og[rows] - ref) ** 2))
+    assert 2.0 < mse[(0, 1.0)] / min(mse[(0, 256.0)], mse[(1, 256.0)]) < 10.5, mse
+    assert mse[(0, 256.0)] / mse[(0, 448.0)] < 0.97, mse
+    assert abs(mse[(1, 256.0)] / mse[(0, 256.0)] - 1) < 0.1, mse
