@@ -73,7 +73,7 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
               kv_order: int = KV_REVERSE, n_sink: int = 0, block_n: int = 0,
               denominator: int = DENOM_FP32_P,
               out_dtype=None, count_collapse: bool = False, per_row: bool = False,
-              out=None, stream=None, host_chunks: int = 8):
+              out=None, stream=None, host_chunks: int = 16):
     """FP8 attention forward.  Returns (O, AttentionStats).
 
     q, k: E4M3 (float8_e4m3fn or uint8 bytes) or both BF16 (the kernel-faithful
