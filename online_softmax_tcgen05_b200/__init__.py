@@ -120,52 +120,91 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     units = [(b, g) for b in range(B) for g in range(H_kv)]       # (batch, kv head)
     nchunk = max(1, min(int(host_chunks), len(units)))
     bounds = [len(units) * i // nchunk for i in range(nchunk + 1)]
-    res = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype,
-                                                  pin_memory=True)
-    compute = torch.cuda.current_stream(dev) if stream is None else stream
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
-    rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
-            if (count_collapse and per_row) else None)
-    keep = []
+    # chunks never cross a batch element, so each piece is one contiguous slice
+    pieces = []
     for c in range(nchunk):
-        u0, u1 = bounds[c], bounds[c + 1]
-        # chunks never cross a batch element, so each is one contiguous slice
-        pieces = []
-        u = u0
-        while u < u1:
+        u = bounds[c]
+        while u < bounds[c + 1]:
             b = units[u][0]
             e = u
-            while e < u1 and units[e][0] == b:
+            while e < bounds[c + 1] and units[e][0] == b:
                 e += 1
             pieces.append((b, units[u][1], units[e - 1][1] + 1))
             u = e
-        for b, g0, g1 in pieces:
-            with torch.cuda.stream(s_in):
-                qd = q[b:b + 1, g0 * group:g1 * group].to(dev, non_blocking=True)
-                kd = k[b:b + 1, g0:g1].to(dev, non_blocking=True)
-                vd = v[b:b + 1, g0:g1].to(dev, non_blocking=True)
-                ev_in = torch.cuda.Event()
-                ev_in.record(s_in)
-            compute.wait_event(ev_in)
-            with torch.cuda.stream(compute):
-                od = torch.empty((1, (g1 - g0) * group, N, d), dtype=out_dtype, device=dev)
-                rd = None if rows is None else rows[b:b + 1, g0 * group:g1 * group]
-                _launch(qd, kd, vd, od, ctr, rd, stream=compute, **kw)
-                ev_c = torch.cuda.Event()
-                ev_c.record(compute)
-            s_out.wait_event(ev_c)
-            with torch.cuda.stream(s_out):
-                res[b:b + 1, g0 * group:g1 * group].copy_(od, non_blocking=True)
-            # the device buffers stay referenced until the output copy has run
-            for t in (qd, kd, vd, od):
-                t.record_stream(s_out)
-                t.record_stream(compute)
-            keep.append((qd, kd, vd, od))
-    s_out.synchronize()
-    compute.wait_stream(s_out)
+    max_g = max(g1 - g0 for _, g0, g1 in pieces)
+    res = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype,
+                                                  pin_memory=True)
+    compute = torch.cuda.current_stream(dev) if stream is None else stream
+    pipe = _host_pipeline(dev)
+    sets = pipe.staging(max_g * group, max_g, N, d, q.dtype, out_dtype)
+    ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
+    rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
+            if (count_collapse and per_row) else None)
+    compute.wait_stream(torch.cuda.current_stream(dev))
+    pipe.s_in.wait_stream(compute)      # earlier work on the caller's stream comes first
+    for i, (b, g0, g1) in enumerate(pieces):
+        nq, nk = (g1 - g0) * group, g1 - g0
+        qb, kb, vb, ob, ev_free = sets[i % 2]
+        qd, kd, vd, od = qb[:, :nq], kb[:, :nk], vb[:, :nk], ob[:, :nq]
+        with torch.cuda.stream(pipe.s_in):
+            if ev_free is not None:
+                pipe.s_in.wait_event(ev_free)   # this set's previous chunk has left the device
+            qd.copy_(q[b:b + 1, g0 * group:g1 * group], non_blocking=True)
+            kd.copy_(k[b:b + 1, g0:g1], non_blocking=True)
+            vd.copy_(v[b:b + 1, g0:g1], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(pipe.s_in)
+        compute.wait_event(ev_in)
+        rd = None if rows is None else rows[b:b + 1, g0 * group:g1 * group]
+        _launch(qd, kd, vd, od, ctr, rd, stream=compute, **kw)
+        ev_c = torch.cuda.Event()
+        ev_c.record(compute)
+        pipe.s_out.wait_event(ev_c)
+        with torch.cuda.stream(pipe.s_out):
+            res[b:b + 1, g0 * group:g1 * group].copy_(od, non_blocking=True)
+            ev_f = torch.cuda.Event()
+            ev_f.record(pipe.s_out)
+        sets[i % 2][4] = ev_f
+    pipe.s_out.synchronize()
+    for st in sets:
+        st[4] = None
     if ctr is not None:
         c = ctr.cpu()
         stats.collapse, stats.collapse_sink_block = int(c[0]), int(c[1])
         stats.collapse_rows = rows
     return res, stats
+
+
+class _HostPipeline:
+    """Per-device copy streams and two sets of device staging buffers for the
+    host-tensor path of attention(), kept across calls so that the steady state
+    allocates nothing.  Not for concurrent use from several host threads."""
+
+    def __init__(self, dev):
+        import torch
+        self.dev = dev
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.key = None
+        self.sets = None
+
+    def staging(self, nq, nk, N, d, qk_dtype, o_dtype):
+        import torch
+        key = (nq, nk, N, d, qk_dtype, o_dtype)
+        if self.key != key:
+            torch.cuda.current_stream(self.dev).synchronize()
+            self.s_out.synchronize()
+            mk = lambda h, dt: torch.empty((1, h, N, d), dtype=dt, device=self.dev)
+            self.sets = [[mk(nq, qk_dtype), mk(nk, qk_dtype), mk(nk, torch.uint8),
+                          mk(nq, o_dtype), None] for _ in range(2)]
+            self.key = key
+        return self.sets
+
+
+_pipelines = {}
+
+
+def _host_pipeline(dev):
+    if dev.index not in _pipelines:
+        _pipelines[dev.index] = _HostPipeline(dev)
+    return _pipelines[dev.index]
