@@ -102,6 +102,11 @@ struct Smem {
   static_assert(BN + D <= (int)TMEM_COLS, "TMEM budget");
 };
 
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
 __device__ __forceinline__ int kv_block_at(int t, int T, int order) {
   return order == FP8ATTN_KV_FORWARD ? t : T - 1 - t;
 }
@@ -336,112 +341,137 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float* s = reinterpret_cast<float*>(sr);
       const bool need_mask = (p.causal && j0 + BN - 1 > q0) || (j0 + BN > p.N);
       const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
-      if (need_mask) {
-#pragma unroll
-        for (int j = 0; j < BN; ++j)
-          if (j0 + j > lim) s[j] = -INFINITY;
-      }
-      // row max: 16 independent chains of three-input max, then a tree
-      float mx16[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) mx16[i] = s[i];
-#pragma unroll
-      for (int j = 16; j + 16 < BN; j += 32)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
-      if constexpr ((BN - 16) % 32 != 0) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
-      }
-      float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
-                       fmax3(mx16[6], mx16[7], mx16[8]));
-      mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
-      mx = fmaxf(mx, mx16[15]);
-      const float m_new = fmaxf(m_run, mx * c);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-      // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
-      float2 acc8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < BN / 2; ++q) {
-        const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
-        if ((q & 7) < POLY_OF_8) {
-          const float2 e = exp2_poly2(y);
-          s[2 * q] = e.x;
-          s[2 * q + 1] = e.y;
-        } else {
-          s[2 * q] = ex2_approx(y.x);
-          s[2 * q + 1] = ex2_approx(y.y);
-        }
-        acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
-      }
-#pragma unroll
-      for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
-      const float rowsum = acc8[0].x + acc8[0].y;
-      if (!p.denom_cast) l = alpha * l + rowsum;
-      // S * p (packed FMUL2), then the E4M3 cast, four keys per word
+      // Most blocks hold no masked key and no sink key and use the FP32 row sum:
+      // they take a copy of the block's arithmetic with no branch in it, so that
+      // the integer work of the cast and the count can interleave with the
+      // exponentials of the same block.
+      const bool plain = !need_mask && j0 >= p.n_sink && !p.denom_cast;
+      float m_new, alpha;
       uint32_t pw[BN / 4];
-      const float2 S2 = make_float2(S, S);
+      auto block_math = [&](auto plain_tag) {
+        constexpr bool PLAIN = decltype(plain_tag)::value;
+        if constexpr (!PLAIN) {
+          if (need_mask) {
 #pragma unroll
-      for (int q = 0; q < BN / 4; ++q) {
-        const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
-        const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
-        pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
-      }
-      if (p.denom_cast) {
-        // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
-        // form a float exactly 2^-120 times the E4M3 value (subnormals included,
-        // as FP32 subnormals); sum those, then scale by 2^120 (exact).
-        float2 d4[4];
+            for (int j = 0; j < BN; ++j)
+              if (j0 + j > lim) s[j] = -INFINITY;
+          }
+        }
+        // row max: 16 independent chains of three-input max, then a tree
+        float mx16[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d4[i] = make_float2(0.f, 0.f);
+        for (int i = 0; i < 16; ++i) mx16[i] = s[i];
+#pragma unroll
+        for (int j = 16; j + 16 < BN; j += 32)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
+        if constexpr ((BN - 16) % 32 != 0) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
+        }
+        float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
+                         fmax3(mx16[6], mx16[7], mx16[8]));
+        mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
+        mx = fmaxf(mx, mx16[15]);
+        m_new = fmaxf(m_run, mx * c);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
+        // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+        float2 acc8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < BN / 2; ++q) {
+          const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
+          if ((q & 7) < POLY_OF_8) {
+            const float2 e = exp2_poly2(y);
+            s[2 * q] = e.x;
+            s[2 * q + 1] = e.y;
+          } else {
+            s[2 * q] = ex2_approx(y.x);
+            s[2 * q + 1] = ex2_approx(y.y);
+          }
+          acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
+        }
+#pragma unroll
+        for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
+        const float rowsum = acc8[0].x + acc8[0].y;
+        if constexpr (PLAIN) {
+          l = alpha * l + rowsum;
+        } else {
+          if (!p.denom_cast) l = alpha * l + rowsum;
+        }
+        // S * p (packed FMUL2), then the E4M3 cast, four keys per word
+        const float2 S2 = make_float2(S, S);
 #pragma unroll
         for (int q = 0; q < BN / 4; ++q) {
-          const uint32_t w = pw[q];
-          const float2 lo = make_float2(__uint_as_float((w & 0x7Fu) << 20),
-                                        __uint_as_float((w & 0x7F00u) << 12));
-          const float2 hi = make_float2(__uint_as_float((w & 0x7F0000u) << 4),
-                                        __uint_as_float((w & 0x7F000000u) >> 4));
-          d4[q & 3] = __fadd2_rn(d4[q & 3], __fadd2_rn(lo, hi));
+          const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
+          const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
+          pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
         }
-        d4[0] = __fadd2_rn(__fadd2_rn(d4[0], d4[1]), __fadd2_rn(d4[2], d4[3]));
-        l = alpha * l + (d4[0].x + d4[0].y) * 0x1p120f;
-      }
-      if constexpr (COUNT) {
-        // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
-        // negative, so byte 0 <=> the cast flushed S*p to zero.  Zero bytes are
-        // found four at a time; blocks that hold a sink or a masked key restrict
-        // the count to the lanes with n_sink <= j <= last visible key.
-        uint32_t zacc = 0;
-        if (j0 >= p.n_sink && !need_mask) {
-          uint32_t z4[4] = {0, 0, 0, 0};
+        if constexpr (!PLAIN) {
+          if (p.denom_cast) {
+            // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
+            // form a float exactly 2^-120 times the E4M3 value (subnormals included,
+            // as FP32 subnormals); sum those, then scale by 2^120 (exact).
+            float2 d4[4];
 #pragma unroll
-          for (int q = 0; q < BN / 4; ++q) {
-            const uint32_t w = pw[q];
-            z4[q & 3] += ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu) >> 7;
-          }
-          zacc = (z4[0] + z4[1]) + (z4[2] + z4[3]);
-        } else {
-          const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);   // block-local
+            for (int i = 0; i < 4; ++i) d4[i] = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int q = 0; q < BN / 4; ++q) {
-            const uint32_t w = pw[q];
-            uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
-            const int a = lo - 4 * q, bq = hi - 4 * q;   // lanes a..bq of this word are valid
-            const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
-            const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
-            zacc += (y & mlo & mhi) >> 7;
+            for (int q = 0; q < BN / 4; ++q) {
+              const uint32_t w = pw[q];
+              const float2 lo = make_float2(__uint_as_float((w & 0x7Fu) << 20),
+                                            __uint_as_float((w & 0x7F00u) << 12));
+              const float2 hi = make_float2(__uint_as_float((w & 0x7F0000u) << 4),
+                                            __uint_as_float((w & 0x7F000000u) >> 4));
+              d4[q & 3] = __fadd2_rn(d4[q & 3], __fadd2_rn(lo, hi));
+            }
+            d4[0] = __fadd2_rn(__fadd2_rn(d4[0], d4[1]), __fadd2_rn(d4[2], d4[3]));
+            l = alpha * l + (d4[0].x + d4[0].y) * 0x1p120f;
           }
         }
-        const uint32_t cblk = (zacc * 0x01010101u) >> 24;   // byte lanes hold <= BN/4 each
-        cnt += cblk;
-        if (j0 < p.n_sink) cnt_sink += cblk;
-      }
+        if constexpr (COUNT) {
+          // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
+          // negative, so byte 0 <=> the cast flushed S*p to zero.
+          uint32_t cblk;
+          if (PLAIN || (j0 >= p.n_sink && !need_mask)) {
+            // Every byte is 0x00..0x7F (sign clear: S*p >= +0; a NaN casts to
+            // 0x7F), so w + 0x7F7F7F7F carries into no neighbour and sets bit 7
+            // of exactly the nonzero bytes; dp4a sums those four flags (x128).
+            uint32_t nz4[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q)
+              nz4[q & 3] = __dp4a((pw[q] + 0x7F7F7F7Fu) & 0x80808080u, 0x01010101u, nz4[q & 3]);
+            cblk = BN - (((nz4[0] + nz4[1]) + (nz4[2] + nz4[3])) >> 7);
+          } else {
+            // blocks that hold a sink or a masked key count only the lanes with
+            // n_sink <= j <= last visible key
+            uint32_t zacc = 0;
+            const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);   // block-local
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q) {
+              const uint32_t w = pw[q];
+              uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
+              const int a = lo - 4 * q, bq = hi - 4 * q;   // lanes a..bq of this word are valid
+              const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
+              const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
+              zacc += (y & mlo & mhi) >> 7;
+            }
+            cblk = (zacc * 0x01010101u) >> 24;   // byte lanes hold <= BN/4 each
+          }
+          cnt += cblk;
+          if constexpr (!PLAIN) {
+            if (j0 < p.n_sink) cnt_sink += cblk;
+          }
+        }
+      };
+      if (plain)
+        block_math(BoolTag<true>{});
+      else
+        block_math(BoolTag<false>{});
       if (t > 0) {
         // P~V(t-1) must be done: it reads the P~ tile and accumulates into O
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE));
