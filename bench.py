@@ -352,7 +352,7 @@ def oracle_sample(W, rows, Q8=None, K8=None, V8=None, cfg=CFG):
     return dt, flops, (Q8, K8, V8)
 
 
-def cpu_baseline(W, cfg=CFG, n_rows=32768):
+def cpu_baseline(W, cfg=CFG, n_rows=65536):
     total = W.B * W.H * W.N
     rows = sample_rows(n_rows, cfg=dict(cfg, H=W.H))
     dt, flops, _ = oracle_sample(W, rows, cfg=cfg)

@@ -20,10 +20,11 @@
 //   warp 5     MMA issuer: S = Q K^T into TMEM (tcgen05 kind::f8f6f4, M=128,
 //              N=block_n, K=32 per instruction), then O += P~ V into TMEM
 //              (V as an MN-major operand).  Owns the TMEM allocation.
-//   warps 0-3  softmax, one thread per query row: tcgen05.ld of its S row, row
-//              max, exp2, FP32 row sum, S-multiply, E4M3 cast into a swizzled
-//              shared-memory P~ tile, collapse count, the O rescale in TMEM when a
-//              row max changed, and the epilogue O / (S l).
+//   warps 0-3  softmax, one thread per query row: tcgen05.ld of its score row,
+//              row max, S*p as one exp2 with log2 S added to the argument, FP32
+//              row sum of S*p, E4M3 cast into a swizzled shared-memory P~ tile,
+//              collapse count, the O rescale in TMEM when a row max changed, and
+//              the epilogue O / l (l: the row sum of S*p, so S divides out).
 // Every mbarrier wait is bounded in time: on expiry the CTA sets a shared
 // abort flag, every role leaves its loop, in-flight copies and MMAs are
 // drained, TMEM is freed and the status word (if given) records where.
@@ -72,7 +73,7 @@ struct KParams {
   int causal, kv_order, n_sink;
   int num_q_tiles;
   float scale_log2;   // scale * log2(e)
-  float S;
+  float log2S;   // log2(S): S*p is taken as 2^(s*c - m + log2 S)
   void* O;
   unsigned long long* ctr;
   unsigned long long* ctr_sink;
@@ -315,7 +316,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     const uint32_t tS = tmem_base + lane_off, tO = tmem_base + lane_off + BN;
     const float c = p.scale_log2;
-    const float S = p.S;
     float m_run = -INFINITY, l = 0.f;
     uint32_t cnt = 0, cnt_sink = 0;
     bool ok = true;
@@ -376,8 +376,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m_new = fmaxf(m_run, mx * c);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-        // p = 2^(s*c - m): packed FFMA2 for the argument, MUFU ex2, split row sums
-        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+        // S*p = 2^(s*c - m + log2 S): packed FFMA2 for the argument, MUFU ex2,
+        // split row sums (of S*p: the epilogue divides by that sum, S included)
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
         float2 acc8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
@@ -404,14 +405,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         } else {
           if (!p.denom_cast) l = alpha * l + rowsum;
         }
-        // S * p (packed FMUL2), then the E4M3 cast, four keys per word
-        const float2 S2 = make_float2(S, S);
+        // the E4M3 cast of S*p, four keys per word
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-          const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), S2);
-          const float2 b2 = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), S2);
-          pw[q] = pack_e4m3x4(a.x, a.y, b2.x, b2.y);
-        }
+        for (int q = 0; q < BN / 4; ++q)
+          pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
         if constexpr (!PLAIN) {
           if (p.denom_cast) {
             // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
@@ -522,7 +519,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     if (ok) {
       tc_fence_after();
-      const float denom = p.denom_cast ? l : S * l;
+      const float denom = l;
       const bool live = row < p.N;
       const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
 #pragma unroll
@@ -772,7 +769,7 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.n_sink = p->n_sink;
   kp.num_q_tiles = (p->N + fp8attn::BM - 1) / fp8attn::BM;
   kp.scale_log2 = p->scale * fp8attn::LOG2E;
-  kp.S = p->S;
+  kp.log2S = (float)std::log2((double)p->S);
   kp.O = p->O;
   kp.ctr = p->collapse_ctr;
   kp.ctr_sink = p->collapse_sink_ctr;

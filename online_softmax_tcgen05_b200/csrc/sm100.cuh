@@ -216,7 +216,13 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
 
 // Four FP32 values -> four E4M3 bytes, element k in byte k.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
-  return cvt_e4m3x2(a1, a0) | (cvt_e4m3x2(a3, a2) << 16);
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return r;
 }
 
 // max of three (sm_100 three-input max)
