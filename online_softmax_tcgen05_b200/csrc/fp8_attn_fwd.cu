@@ -324,10 +324,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t prow = sP + (r >> 3) * (8 * BN) + (r & 7) * BN;
     const uint32_t pswz = (BN == 128) ? (uint32_t)(r & 7) : (uint32_t)((r & 7) >> 1);
 
-    for (int t = 0; t < T; ++t) {
+    // S(0) here; S(t+1) at the end of block t (see below)
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, 0, ctl, WAIT_SM_S_FULL));
+    for (int t = 0; ok && t < T; ++t) {
       const int j0 = kv_block_at(t, T, p.kv_order) * BN;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, t & 1, ctl, WAIT_SM_S_FULL));
-      if (!ok) break;
       tc_fence_after();
       uint32_t sr[BN];
 #pragma unroll
@@ -469,12 +469,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         block_math(BoolTag<true>{});
       else
         block_math(BoolTag<false>{});
-      if (t > 0) {
-        // P~V(t-1) must be done: it reads the P~ tile and accumulates into O
+      // P~V(t-1) must be done before the P~ tile is rewritten and O rescaled.  The
+      // commit that completes S(t+1) tracks every MMA issued before QK^T(t+1),
+      // P~V(t-1) among them, so one wait serves both this block's hand-off and
+      // the next block's scores; the last block waits for P~V(t-1) itself.
+      if (t + 1 < T) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, (t + 1) & 1, ctl, WAIT_SM_S_FULL));
+        if (!ok) break;
+      } else if (t > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, ctl, WAIT_SM_O_DONE));
         if (!ok) break;
-        tc_fence_after();
       }
+      tc_fence_after();
 #pragma unroll
       for (int q = 0; q < BN / 16; ++q) {
         const uint32_t dst = prow + ((q ^ pswz) << 4);
