@@ -325,7 +325,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(W, cfg, n_rows=8192 if strong else 32768)
+        line["cpu_baseline"] = cpu_baseline(W, cfg, n_rows=8192 if strong else 65536)
     return line
 
 

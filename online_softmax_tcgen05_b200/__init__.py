@@ -80,9 +80,12 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     mode: QK^T on BF16 operands, P~ and V in E4M3); v: E4M3.
 
     Host (CPU) tensors: the work is cut into up to ``host_chunks`` pieces along
-    the (batch, kv-head) axis; the copy of piece g+1 to the device runs on its
-    own stream while piece g computes, and piece g's output returns on a third
-    stream.  Pinned host memory makes those copies asynchronous."""
+    the (batch, kv-head) axis.  The copy of piece g+1 to the device runs on its
+    own stream while piece g computes, and piece g's output returns on another.
+    Consecutive pieces compute on two alternating streams, so that one piece's
+    kernel can fill the SMs that the previous piece's last wave leaves idle.
+    Pinned host memory makes the copies asynchronous.  ``stream`` (default: the
+    current stream) is ordered before and after the whole call."""
     import torch
     q, k, v = _as_bytes(q, True), _as_bytes(k, True), _as_bytes(v)
     if (q.dtype == torch.bfloat16) != (k.dtype == torch.bfloat16):
@@ -134,17 +137,21 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     max_g = max(g1 - g0 for _, g0, g1 in pieces)
     res = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype,
                                                   pin_memory=True)
-    compute = torch.cuda.current_stream(dev) if stream is None else stream
+    caller = torch.cuda.current_stream(dev) if stream is None else stream
     pipe = _host_pipeline(dev)
     sets = pipe.staging(max_g * group, max_g, N, d, q.dtype, out_dtype)
+    ns = len(sets)
     ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
     rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
             if (count_collapse and per_row) else None)
-    compute.wait_stream(torch.cuda.current_stream(dev))
-    pipe.s_in.wait_stream(compute)      # earlier work on the caller's stream comes first
+    cur = torch.cuda.current_stream(dev)   # the counters were zeroed on it
+    pipe.s_in.wait_stream(caller)       # earlier work on the caller's stream comes first
+    for sc in pipe.s_comp:
+        sc.wait_stream(caller)
+        sc.wait_stream(cur)
     for i, (b, g0, g1) in enumerate(pieces):
         nq, nk = (g1 - g0) * group, g1 - g0
-        qb, kb, vb, ob, ev_free = sets[i % 2]
+        qb, kb, vb, ob, ev_free = sets[i % ns]
         qd, kd, vd, od = qb[:, :nq], kb[:, :nk], vb[:, :nk], ob[:, :nq]
         with torch.cuda.stream(pipe.s_in):
             if ev_free is not None:
@@ -154,6 +161,7 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
             vd.copy_(v[b:b + 1, g0:g1], non_blocking=True)
             ev_in = torch.cuda.Event()
             ev_in.record(pipe.s_in)
+        compute = pipe.s_comp[i % 2]
         compute.wait_event(ev_in)
         rd = None if rows is None else rows[b:b + 1, g0 * group:g1 * group]
         _launch(qd, kd, vd, od, ctr, rd, stream=compute, **kw)
@@ -164,8 +172,9 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
             res[b:b + 1, g0 * group:g1 * group].copy_(od, non_blocking=True)
             ev_f = torch.cuda.Event()
             ev_f.record(pipe.s_out)
-        sets[i % 2][4] = ev_f
+        sets[i % ns][4] = ev_f
     pipe.s_out.synchronize()
+    caller.wait_stream(pipe.s_out)
     for st in sets:
         st[4] = None
     if ctr is not None:
@@ -176,27 +185,36 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
 
 
 class _HostPipeline:
-    """Per-device copy streams and two sets of device staging buffers for the
-    host-tensor path of attention(), kept across calls so that the steady state
-    allocates nothing.  Not for concurrent use from several host threads."""
+    """Per-device copy and compute streams and ``nsets`` sets of device staging
+    buffers for the host-tensor path of attention(), kept across calls so that
+    the steady state allocates nothing.  A set is reused by the piece ``nsets``
+    places later, whose upload therefore waits for this piece's download: with
+    two sets each piece would cost a download plus an upload.  Not for
+    concurrent use from several host threads."""
+
+    nsets = 3
 
     def __init__(self, dev):
         import torch
         self.dev = dev
         self.s_in = torch.cuda.Stream(dev)
         self.s_out = torch.cuda.Stream(dev)
+        self.s_comp = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
         self.key = None
         self.sets = None
 
     def staging(self, nq, nk, N, d, qk_dtype, o_dtype):
         import torch
-        key = (nq, nk, N, d, qk_dtype, o_dtype)
+        key = (nq, nk, N, d, qk_dtype, o_dtype, self.nsets)
         if self.key != key:
             torch.cuda.current_stream(self.dev).synchronize()
+            for st in self.s_comp:
+                st.synchronize()
             self.s_out.synchronize()
             mk = lambda h, dt: torch.empty((1, h, N, d), dtype=dt, device=self.dev)
+            self.sets = None   # free the old buffers before allocating new ones
             self.sets = [[mk(nq, qk_dtype), mk(nk, qk_dtype), mk(nk, torch.uint8),
-                          mk(nq, o_dtype), None] for _ in range(2)]
+                          mk(nq, o_dtype), None] for _ in range(self.nsets)]
             self.key = key
         return self.sets
 
