@@ -97,6 +97,34 @@ def peak_tflops():
         return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2"
 
 
+def fp8_gemm_peak(dev, n=8192, reps=10):
+    """This GPU's dense FP8 GEMM rate in TFLOP/s: torch._scaled_mm (cuBLASLt) on
+    E4M3 n x n x n with unit scales, BF16 out, best of `reps` CUDA-event timings.
+    A context denominator beside the roofline's peak; None where unsupported."""
+    import torch
+    try:
+        g = torch.Generator(device=dev).manual_seed(7)
+        a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        bt = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        run = lambda: torch._scaled_mm(a, bt, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, bt
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
 KERNEL_SOURCES = ["online_softmax_tcgen05_b200/csrc/fp8_attn_fwd.cu",
                   "online_softmax_tcgen05_b200/csrc/sm100.cuh",
                   "online_softmax_tcgen05_b200/csrc/exp2_poly.cuh"]
@@ -294,6 +322,7 @@ def run_ours(args, rank, world, local_rank):
 
     if rank != 0:
         return None
+    fp8_gemm = fp8_gemm_peak(dev)   # after every timed region
     import oracle
     pairs = world * B * H * (N - cfg["n_sink"]) * (N - cfg["n_sink"] + 1) // 2
     frac = collapse_total / args.steps / pairs
@@ -309,7 +338,12 @@ def run_ours(args, rank, world, local_rank):
                     "l2": "inputs 201 MB > 126 MB L2, no flush"}),
         "value_counter_off": round(job_tflops(flops, world, ms_off / args.steps), 2),
         "pct_of_fp8_peak": {"measured": round(kernel_tflops / peak, 4),
-                            "nominal_4500": round(kernel_tflops / 4500.0, 4)},
+                            "nominal_4500": round(kernel_tflops / 4500.0, 4),
+                            "fp8_gemm_this_gpu": (None if fp8_gemm is None else
+                                                  {"tflops": round(fp8_gemm, 1),
+                                                   "frac": round(kernel_tflops / fp8_gemm, 4),
+                                                   "how": "torch._scaled_mm E4M3 8192^3, "
+                                                          "best of 10"})},
         "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2),
                      "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(kernel_tflops / peak, 4), "traffic": measured_traffic(),
