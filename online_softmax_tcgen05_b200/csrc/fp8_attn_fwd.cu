@@ -541,7 +541,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     if (ok) {
       tc_fence_after();
-      const float denom = l;
+      // O = acc * 1/l, l being the row sum of S*p (so S divides out here); one
+      // correctly rounded reciprocal per row, then a multiply per element
+      const float inv_l = __frcp_rn(l);
       const bool live = row < p.N;
       const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
 #pragma unroll
@@ -551,7 +553,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_wait_ld();
         float v[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), denom);
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * inv_l;
         if (live) {
           if constexpr (OUT_BF16) {
             uint32_t w[16];
