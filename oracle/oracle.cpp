@@ -195,9 +195,10 @@ int oracle_attn_exact(const void* Q, const void* K, const uint8_t* V,
     if (H % Hkv) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
-    if (nthreads > 0) omp_set_num_threads(nthreads);
+    // nthreads applies to this call only (0: every processor)
+    const int nt = nthreads > 0 ? nthreads : omp_get_num_procs();
     const int group = H / Hkv;
-    #pragma omp parallel
+    #pragma omp parallel num_threads(nt)
     {
         std::vector<double> s(N), q(d), acc(d);
         #pragma omp for schedule(dynamic, 4)
@@ -262,11 +263,12 @@ int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
     if (H % Hkv || block_n <= 0) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
-    if (nthreads > 0) omp_set_num_threads(nthreads);
+    // nthreads applies to this call only (0: every processor)
+    const int nt = nthreads > 0 ? nthreads : omp_get_num_procs();
     const int group = H / Hkv;
     const int nblocks = (N + block_n - 1) / block_n;
     uint64_t tot_sink = 0, tot_other = 0;
-    #pragma omp parallel reduction(+ : tot_sink, tot_other)
+    #pragma omp parallel num_threads(nt) reduction(+ : tot_sink, tot_other)
     {
         std::vector<float> q(d), acc(d), s(block_n), vdec((size_t)block_n * d);
         std::vector<uint8_t> pt(block_n);
@@ -333,10 +335,11 @@ int oracle_collapse_logits(const float* logits, int64_t nrows, int N, int block_
                            float S, int kv_order, uint32_t* collapse_rows,
                            uint64_t* collapse_totals, int nthreads) {
     if (block_n <= 0) return -1;
-    if (nthreads > 0) omp_set_num_threads(nthreads);
+    // nthreads applies to this call only (0: every processor)
+    const int nt = nthreads > 0 ? nthreads : omp_get_num_procs();
     const int nblocks = (N + block_n - 1) / block_n;
     uint64_t tot_sink = 0, tot_other = 0;
-    #pragma omp parallel reduction(+ : tot_sink, tot_other)
+    #pragma omp parallel num_threads(nt) reduction(+ : tot_sink, tot_other)
     {
         std::vector<uint8_t> pt(block_n);
         #pragma omp for schedule(static)
