@@ -105,6 +105,7 @@ CASES = [
     (1, 4, 2, 700, 64, 128, 1),
     (1, 1, 1, 333, 64, 64, 1),
     (1, 1, 1, 256, 128, 64, 0),
+    (2, 4, 2, 700, 64, 128, 1),   # causal CTA order across two batch elements
 ]
 
 
