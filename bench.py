@@ -140,10 +140,12 @@ def kernel_sources_sha256():
     return h.hexdigest()
 
 
-def measured_traffic():
+def measured_traffic(prefill=True):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-    the committed ncu capture of this workload, or None when the kernel sources
-    changed since that capture."""
+    the committed ncu capture of the prefill workload; None for another workload
+    or when the kernel sources changed since that capture."""
+    if not prefill:
+        return None
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
@@ -346,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
                                                           "best of 10"})},
         "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2),
                      "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(kernel_tflops / peak, 4), "traffic": measured_traffic(),
+                     "frac": round(kernel_tflops / peak, 4), "traffic": measured_traffic(prefill=not strong),
                      "peak_source": peak_src + " (of measured)" if "measured" in peak_src
                      else peak_src},
         "collapse": {"fraction": frac, "count_per_step": collapse_total // args.steps // world,
