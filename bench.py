@@ -97,6 +97,19 @@ def peak_tflops():
         return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2"
 
 
+# E[max of k independent standard normals], for k sink keys (1/sqrt(pi) at k = 2)
+EXPECTED_MAX_NORMAL = {1: 0.0, 2: 0.5641895835, 3: 0.8462843753, 4: 1.0293753730}
+
+
+def closed_form_F(delta, S, k=4):
+    """The P-cast paper's closed form for the forward-order fraction of non-sink
+    probabilities that the E4M3 cast flushes to zero (Methodology, theoretical
+    framework): F(Delta, S) = Phi(Delta + delta_k - 10 ln 2 - ln S).  A reported
+    reference value beside the measured fraction."""
+    x = delta + EXPECTED_MAX_NORMAL[k] - 10.0 * math.log(2.0) - math.log(S)
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
 def fp8_gemm_peak(dev, n=8192, reps=10):
     """This GPU's dense FP8 GEMM rate in TFLOP/s: torch._scaled_mm (cuBLASLt) on
     E4M3 n x n x n with unit scales, BF16 out, best of `reps` CUDA-event timings.
@@ -325,7 +338,6 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
     fp8_gemm = fp8_gemm_peak(dev)   # after every timed region
-    import oracle
     pairs = world * B * H * (N - cfg["n_sink"]) * (N - cfg["n_sink"] + 1) // 2
     frac = collapse_total / args.steps / pairs
     line = {
@@ -353,8 +365,7 @@ def run_ours(args, rank, world, local_rank):
                      else peak_src},
         "collapse": {"fraction": frac, "count_per_step": collapse_total // args.steps // world,
                      "in_sink_block": collapse_sink // args.steps // world,
-                     "closed_form_forward_F": oracle.underflow_fraction_closed(cfg["delta"],
-                                                                               cfg["S"])},
+                     "closed_form_forward_F": closed_form_F(cfg["delta"], cfg["S"], cfg["n_sink"])},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / e2e_steps, 3)},
         "gpu_launches": args.steps,
@@ -431,6 +442,165 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------ reports --
+# `--report collapse` and `--report configs` (one GPU): one JSON line per run,
+# for the record of the method's evaluation; the default bench line above is
+# unaffected.
+class _ReportLaunch:
+    """One configuration on device inputs, with its buffers allocated once:
+    launch() only enqueues the kernel (for timing); counts() zeroes the
+    counters, runs once and returns (collapse total, in sink-holding blocks)."""
+
+    def __init__(self, fa, ins, shape, causal, S, order, n_sink, count=True):
+        import torch
+        self.fa, (self.q, self.k, self.v) = fa, ins
+        self.shape, self.causal, self.S, self.order, self.ns = shape, causal, S, order, n_sink
+        B, H, Hkv, N, d = shape
+        self.O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=self.q.device)
+        self.ctr = torch.zeros(2, dtype=torch.int64, device=self.q.device) if count else None
+
+    def launch(self):
+        B, H, Hkv, N, d = self.shape
+        c = self.ctr
+        self.fa.fp8_attn_fwd_ex(self.q, self.k, self.v, self.O, B=B, H=H, H_kv=Hkv, N=N, d=d,
+                                causal=bool(self.causal), scale=1.0 / math.sqrt(d), S=self.S,
+                                kv_order=self.order, n_sink=self.ns, o_dtype=self.fa.O_BF16,
+                                block_n=128, collapse_ctr=None if c is None else c[0:1],
+                                collapse_sink_ctr=None if c is None else c[1:2])
+
+    def counts(self):
+        import torch
+        self.ctr.zero_()
+        self.launch()
+        torch.cuda.synchronize()
+        c = self.ctr.cpu().tolist()
+        return int(c[0]), int(c[1])
+
+
+def _median_ms(fn, reps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def _visible_pairs(B, H, N, n_sink, causal):
+    """Non-sink (query, key) pairs the collapse fraction is taken over."""
+    m = N - n_sink
+    return B * H * (m * (m + 1) // 2 if causal else N * m)
+
+
+def report_collapse(dev):
+    """Delta/S sweep (B1 H8 N4096 d128, non-causal, 4 sink keys): the measured
+    collapse fraction in forward order beside the closed form F(Delta, S), and the
+    fraction outside the sink-holding KV block in reverse order."""
+    import torch
+    import workload
+    import online_softmax_tcgen05_b200 as fa
+    B, H, N, d, ns = 1, 8, 4096, 128, 4
+    pairs = _visible_pairs(B, H, N, ns, 0)
+    for delta in range(0, 13):
+        W = workload.make_sink_workload(B, H, H, N, d, ns, float(delta),
+                                        seed=workload.CONFIG_SEED_BASE + 2)
+        ins = [fa.e4m3_cast(torch.from_numpy(x).to(dev)) for x in (W.q, W.k, W.v)]
+        for S in (1.0, 16.0, 256.0, 448.0):
+            line = {"report": "collapse", "workload": "sweep B1 H8 N4096 d128 non-causal, "
+                    "4 sink keys", "delta": delta, "S": S,
+                    "closed_form_F": round(closed_form_F(delta, S, ns), 6)}
+            for order, name in ((fa.KV_FORWARD, "forward"), (fa.KV_REVERSE, "reverse")):
+                tot, sink = _ReportLaunch(fa, ins, (B, H, H, N, d), 0, S, order, ns).counts()
+                line[name] = {"fraction": round(tot / pairs, 6),
+                              "outside_sink_block": round((tot - sink) / pairs, 8)}
+            print(json.dumps(line), flush=True)
+        del ins
+
+
+def report_configs(dev):
+    """The timing protocols of the evaluation's larger configurations (median of
+    CUDA-event timings), with the collapse fraction of each run: the causal GQA
+    prefill with the counter on and off; batched non-causal with forward and
+    reverse order alternating; the long-context causal GQA grid Delta x S x order."""
+    import torch
+    import workload
+    import online_softmax_tcgen05_b200 as fa
+
+    def gen(B, H, Hkv, N, d, ns, delta, seed):
+        W = workload.make_sink_workload(B, H, Hkv, N, d, ns, delta, seed=seed)
+        return [fa.e4m3_cast(torch.from_numpy(x).to(dev)) for x in (W.q, W.k, W.v)]
+
+    def launch(ins, shape, causal, S, order, ns, count):
+        return _ReportLaunch(fa, ins, shape, causal, S, order, ns, count)
+
+    # prefill: B1 H32/8 N32768, causal, Delta 8, S 256, reverse; 10 warm-up, median of 50
+    shape = (1, 32, 8, 32768, 128)
+    ins = gen(*shape, 4, 8.0, workload.CONFIG_SEED_BASE + 3)
+    flops = algorithmic_flops(1, 32, 32768, 128, True)
+    for count in (True, False):
+        ms = _median_ms(launch(ins, shape, 1, 256.0, fa.KV_REVERSE, 4, count).launch, 50, 10)
+        print(json.dumps({"report": "configs", "workload": "prefill B1 H32/8 N32768 d128 causal",
+                          "S": 256.0, "order": "reverse", "counter": count,
+                          "median_ms": round(ms, 4), "TFLOP/s": round(flops / ms / 1e9, 1)}),
+              flush=True)
+    del ins
+    # batched: B4 H32 N8192, non-causal, Delta 10, S 256; forward and reverse alternating
+    shape = (4, 32, 32, 8192, 128)
+    ins = gen(*shape, 4, 10.0, workload.CONFIG_SEED_BASE + 4)
+    flops = algorithmic_flops(4, 32, 8192, 128, False)
+    runs = {fa.KV_FORWARD: launch(ins, shape, 0, 256.0, fa.KV_FORWARD, 4, True),
+            fa.KV_REVERSE: launch(ins, shape, 0, 256.0, fa.KV_REVERSE, 4, True)}
+    times = {fa.KV_FORWARD: [], fa.KV_REVERSE: []}
+    for _ in range(5):
+        for o in runs:
+            runs[o].launch()
+    torch.cuda.synchronize()
+    for _ in range(50):
+        for o in runs:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            runs[o].launch()
+            e1.record()
+            torch.cuda.synchronize()
+            times[o].append(e0.elapsed_time(e1))
+    for o, name in ((fa.KV_FORWARD, "forward"), (fa.KV_REVERSE, "reverse")):
+        tot, sink = runs[o].counts()
+        ms = statistics.median(times[o])
+        print(json.dumps({"report": "configs", "workload": "batched B4 H32 N8192 d128 non-causal",
+                          "S": 256.0, "delta": 10.0, "order": name, "counter": True,
+                          "median_ms": round(ms, 4), "TFLOP/s": round(flops / ms / 1e9, 1),
+                          "collapse_fraction": tot / _visible_pairs(4, 32, 8192, 4, 0)}),
+              flush=True)
+    del ins, runs
+    # long context: B1 H32/8 N131072, causal, counter on; Delta {6, 10} x S {1, 256} x order
+    shape = (1, 32, 8, 131072, 128)
+    flops = algorithmic_flops(1, 32, 131072, 128, True)
+    pairs = _visible_pairs(1, 32, 131072, 4, 1)
+    for delta in (6.0, 10.0):
+        ins = gen(*shape, 4, delta, workload.CONFIG_SEED_BASE + 5)
+        for S in (1.0, 256.0):
+            for o, name in ((fa.KV_REVERSE, "reverse"), (fa.KV_FORWARD, "forward")):
+                run = launch(ins, shape, 1, S, o, 4, True)
+                ms = _median_ms(run.launch, 3, 1)
+                tot, sink = run.counts()
+                print(json.dumps({"report": "configs",
+                                  "workload": "long B1 H32/8 N131072 d128 causal",
+                                  "delta": delta, "S": S, "order": name, "counter": True,
+                                  "median_ms": round(ms, 3), "TFLOP/s": round(flops / ms / 1e9, 1),
+                                  "collapse_fraction": tot / pairs,
+                                  "outside_sink_block": (tot - sink) / pairs,
+                                  "closed_form_F": round(closed_form_F(delta, S, 4), 8)}),
+                      flush=True)
+        del ins
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -443,7 +613,16 @@ def main():
                          "the long-context problem split by kv heads (strong scaling)")
     ap.add_argument("--mode", choices=["full", "kernel"], default="full",
                     help="kernel: only the device-timed kernel loop (for profiling)")
+    ap.add_argument("--report", choices=["collapse", "configs"], default=None,
+                    help="one GPU: JSON lines for the Delta/S collapse sweep against the closed "
+                         "form, or the timing protocols of the larger configurations")
     args = ap.parse_args()
+    if args.report is not None:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        (report_collapse if args.report == "collapse" else report_configs)(dev)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
