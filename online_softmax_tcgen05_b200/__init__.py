@@ -149,27 +149,41 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     for sc in pipe.s_comp:
         sc.wait_stream(caller)
         sc.wait_stream(cur)
+    step = 0   # sub-steps alternate between the two compute streams
     for i, (b, g0, g1) in enumerate(pieces):
         nq, nk = (g1 - g0) * group, g1 - g0
         qb, kb, vb, ob, ev_free = sets[i % ns]
         qd, kd, vd, od = qb[:, :nq], kb[:, :nk], vb[:, :nk], ob[:, :nq]
+        hq = g0 * group
+        # The first piece's upload and the last piece's download overlap no
+        # compute.  A first or last piece of one kv head therefore runs as one
+        # kernel per query head, K and V uploaded once: each head's kernel waits
+        # only for its own Q, and each head's O returns as soon as it is done.
+        split = nk == 1 and group > 1 and len(pieces) > 1 and i in (0, len(pieces) - 1)
+        subs = [(j, j + 1) for j in range(nq)] if split else [(0, nq)]
         with torch.cuda.stream(pipe.s_in):
             if ev_free is not None:
                 pipe.s_in.wait_event(ev_free)   # this set's previous chunk has left the device
-            qd.copy_(q[b:b + 1, g0 * group:g1 * group], non_blocking=True)
             kd.copy_(k[b:b + 1, g0:g1], non_blocking=True)
             vd.copy_(v[b:b + 1, g0:g1], non_blocking=True)
-            ev_in = torch.cuda.Event()
-            ev_in.record(pipe.s_in)
-        compute = pipe.s_comp[i % 2]
-        compute.wait_event(ev_in)
-        rd = None if rows is None else rows[b:b + 1, g0 * group:g1 * group]
-        _launch(qd, kd, vd, od, ctr, rd, stream=compute, **kw)
-        ev_c = torch.cuda.Event()
-        ev_c.record(compute)
-        pipe.s_out.wait_event(ev_c)
+            ev_in = []
+            for a0, a1 in subs:
+                qd[:, a0:a1].copy_(q[b:b + 1, hq + a0:hq + a1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(pipe.s_in)
+                ev_in.append(ev)
+        for (a0, a1), ev in zip(subs, ev_in):
+            compute = pipe.s_comp[step % 2]
+            step += 1
+            compute.wait_event(ev)
+            rd = None if rows is None else rows[b:b + 1, hq + a0:hq + a1]
+            _launch(qd[:, a0:a1], kd, vd, od[:, a0:a1], ctr, rd, stream=compute, **kw)
+            ev_c = torch.cuda.Event()
+            ev_c.record(compute)
+            pipe.s_out.wait_event(ev_c)
+            with torch.cuda.stream(pipe.s_out):
+                res[b:b + 1, hq + a0:hq + a1].copy_(od[:, a0:a1], non_blocking=True)
         with torch.cuda.stream(pipe.s_out):
-            res[b:b + 1, g0 * group:g1 * group].copy_(od, non_blocking=True)
             ev_f = torch.cuda.Event()
             ev_f.record(pipe.s_out)
         sets[i % ns][4] = ev_f
