@@ -393,7 +393,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
         // S*p = 2^(s*c - m + log2 S): packed FFMA2 for the argument, MUFU ex2,
-        // split row sums (of S*p: the epilogue divides by that sum, S included)
+        // split row sums (of S*p: the epilogue scales O by 1 / that sum, S included)
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
         float2 acc8[8];
 #pragma unroll
