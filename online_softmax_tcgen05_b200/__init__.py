@@ -173,7 +173,7 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
                 ev.record(pipe.s_in)
                 ev_in.append(ev)
         for (a0, a1), ev in zip(subs, ev_in):
-            compute = pipe.s_comp[step % 2]
+            compute = pipe.s_comp[step % len(pipe.s_comp)]
             step += 1
             compute.wait_event(ev)
             rd = None if rows is None else rows[b:b + 1, hq + a0:hq + a1]
