@@ -601,6 +601,39 @@ def report_configs(dev):
         del ins
 
 
+def report_batched_orders(dev):
+    """Batched non-causal configuration (B4 H32 N8192 d128, Delta 10, S 256, counter
+    on): forward and reverse KV order, 3 warm-up pairs then 10 alternating timed
+    pairs (launches 7 and 8 are the first timed forward and reverse ones, for a
+    profiler capture)."""
+    import torch
+    import workload
+    import online_softmax_tcgen05_b200 as fa
+    shape = (4, 32, 32, 8192, 128)
+    W = workload.make_sink_workload(*shape, 4, 10.0, seed=workload.CONFIG_SEED_BASE + 4)
+    ins = [fa.e4m3_cast(torch.from_numpy(x).to(dev)) for x in (W.q, W.k, W.v)]
+    runs = [(name, _ReportLaunch(fa, ins, shape, 0, 256.0, o, 4, True))
+            for name, o in (("forward", fa.KV_FORWARD), ("reverse", fa.KV_REVERSE))]
+    for _ in range(3):
+        for _, r in runs:
+            r.launch()
+    torch.cuda.synchronize()
+    times = {name: [] for name, _ in runs}
+    for _ in range(10):
+        for name, r in runs:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            r.launch()
+            e1.record()
+            torch.cuda.synchronize()
+            times[name].append(e0.elapsed_time(e1))
+    flops = algorithmic_flops(4, 32, 8192, 128, False)
+    for name, _ in runs:
+        ms = statistics.median(times[name])
+        print(json.dumps({"report": "batched-orders", "order": name, "median_ms": round(ms, 4),
+                          "TFLOP/s": round(flops / ms / 1e9, 1)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -613,7 +646,7 @@ def main():
                          "the long-context problem split by kv heads (strong scaling)")
     ap.add_argument("--mode", choices=["full", "kernel"], default="full",
                     help="kernel: only the device-timed kernel loop (for profiling)")
-    ap.add_argument("--report", choices=["collapse", "configs"], default=None,
+    ap.add_argument("--report", choices=["collapse", "configs", "batched-orders"], default=None,
                     help="one GPU: JSON lines for the Delta/S collapse sweep against the closed "
                          "form, or the timing protocols of the larger configurations")
     args = ap.parse_args()
@@ -621,7 +654,8 @@ def main():
         import torch
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
-        (report_collapse if args.report == "collapse" else report_configs)(dev)
+        {"collapse": report_collapse, "configs": report_configs,
+         "batched-orders": report_batched_orders}[args.report](dev)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
