@@ -121,6 +121,14 @@ typedef struct {
                                             (1-based), so the MMA warp's bounded wait runs
                                             out, status_word records it and the launch ends
                                             with O incomplete */
+  int q_begin, q_end;     /* query rows [q_begin, q_end) of every (batch, head) plane are
+                             computed; O rows, per-row counts and collapse counts of the
+                             other rows are left untouched.  q_begin = q_end = 0 selects
+                             all N rows.  Otherwise 0 <= q_begin < q_end <= N, q_begin a
+                             multiple of 128 (the query tile), q_end a multiple of 128 or
+                             N.  Causal rows see keys 0 .. row whatever the range, so a
+                             problem can be computed as several launches over disjoint
+                             ranges (short causal tiles last, for instance). */
 } fp8attn_params;
 
 int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream);

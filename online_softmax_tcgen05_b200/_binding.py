@@ -37,7 +37,8 @@ class Params(ctypes.Structure):
                 ("qk_dtype", ctypes.c_int), ("denominator", ctypes.c_int),
                 ("collapse_ctr", ctypes.c_void_p), ("collapse_sink_ctr", ctypes.c_void_p),
                 ("collapse_rows", ctypes.c_void_p), ("status_word", ctypes.c_void_p),
-                ("timeout_ns", ctypes.c_ulonglong), ("debug_skip_kv_step", ctypes.c_int)]
+                ("timeout_ns", ctypes.c_ulonglong), ("debug_skip_kv_step", ctypes.c_int),
+                ("q_begin", ctypes.c_int), ("q_end", ctypes.c_int)]
 
 
 # exported symbol -> (argtypes, restype); every symbol of include/fp8attn.h
@@ -124,8 +125,11 @@ def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S
                     kv_order=KV_REVERSE, n_sink=0, o_dtype=O_BF16, block_n=0, denominator=0,
                     qk_dtype=QK_E4M3,
                     collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None,
-                    status_word=None, timeout_ns=0, debug_skip_kv_step=0, stream=None):
-    """Full-parameter entry point (all tensors on the device)."""
+                    status_word=None, timeout_ns=0, debug_skip_kv_step=0, q_begin=0, q_end=0,
+                    stream=None):
+    """Full-parameter entry point (all tensors on the device).  ``q_begin``,
+    ``q_end``: the query-row range of each (batch, head) plane to compute
+    (0, 0 = all rows)."""
     p = Params(Q=Q.data_ptr(), K=K.data_ptr(), V=V.data_ptr(), O=O.data_ptr(),
                B=B, H=H, H_kv=H_kv, N=N, d=d, causal=int(causal),
                scale=float(scale if scale is not None else 1.0 / math.sqrt(d)), S=float(S),
@@ -135,5 +139,6 @@ def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S
                collapse_sink_ctr=None if collapse_sink_ctr is None else collapse_sink_ctr.data_ptr(),
                collapse_rows=None if collapse_rows is None else collapse_rows.data_ptr(),
                status_word=None if status_word is None else status_word.data_ptr(),
-               timeout_ns=int(timeout_ns), debug_skip_kv_step=int(debug_skip_kv_step))
+               timeout_ns=int(timeout_ns), debug_skip_kv_step=int(debug_skip_kv_step),
+               q_begin=int(q_begin), q_end=int(q_end))
     _check(load_library().fp8_attn_fwd_ex(ctypes.byref(p), _stream(stream)), "fp8_attn_fwd_ex")

@@ -71,7 +71,8 @@ enum : uint32_t {
 struct KParams {
   int B, H, Hkv, N, group;
   int causal, kv_order, n_sink;
-  int num_q_tiles;
+  int tile0;          // first query tile of the launch (q_begin / 128)
+  int num_q_tiles;    // query tiles in the launch
   int sched_group;    // (batch, head) planes per causal scheduling group; divides B * H
   float scale_log2;   // scale * log2(e)
   float log2S;   // log2(S): S*p is taken as 2^(s*c - m + log2 S)
@@ -153,10 +154,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int lin = (int)blockIdx.y * (int)gridDim.x + (int)blockIdx.x;
     const int per_group = p.num_q_tiles * p.sched_group;
     const int g = lin / per_group, inner = lin % per_group;
-    tile = p.num_q_tiles - 1 - inner / p.sched_group;
+    tile = p.tile0 + p.num_q_tiles - 1 - inner / p.sched_group;
     bh = g * p.sched_group + inner % p.sched_group;
   } else {
-    tile = (int)blockIdx.x;
+    tile = p.tile0 + (int)blockIdx.x;
     bh = (int)blockIdx.y;
   }
   const int h = bh % p.H, b = bh / p.H;
@@ -701,7 +702,7 @@ cudaError_t launch_dt(bool bf16, bool count, bool qk_bf16, const CUtensorMap& q,
 
 extern "C" {
 
-int fp8attn_version(void) { return 100; }
+int fp8attn_version(void) { return 101; }
 
 size_t fp8attn_params_sizeof(void) { return sizeof(fp8attn_params); }
 
@@ -764,6 +765,13 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
     return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
   if ((long long)p->B * p->H > 65535LL * 65535LL) return fail(FP8ATTN_EINVAL, "B*H too large");
+  const bool all_rows = p->q_begin == 0 && p->q_end == 0;
+  if (!all_rows) {
+    if (p->q_begin < 0 || p->q_end > p->N || p->q_begin >= p->q_end)
+      return fail(FP8ATTN_EINVAL, "q_begin, q_end must satisfy 0 <= q_begin < q_end <= N");
+    if (p->q_begin % fp8attn::BM || (p->q_end % fp8attn::BM && p->q_end != p->N))
+      return fail(FP8ATTN_EINVAL, "q_begin must be a multiple of 128, q_end a multiple of 128 or N");
+  }
   if ((long long)p->B * p->H * p->N == 0) return FP8ATTN_OK;   // nothing to compute
   if (!p->Q || !p->K || !p->V || !p->O) return fail(FP8ATTN_EINVAL, "Q, K, V, O must be non-NULL");
   if (!aligned16(p->Q) || !aligned16(p->K) || !aligned16(p->V) || !aligned16(p->O))
@@ -803,7 +811,11 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.causal = p->causal;
   kp.kv_order = p->kv_order;
   kp.n_sink = p->n_sink;
-  kp.num_q_tiles = (p->N + fp8attn::BM - 1) / fp8attn::BM;
+  {
+    const int r0 = all_rows ? 0 : p->q_begin, r1 = all_rows ? p->N : p->q_end;
+    kp.tile0 = r0 / fp8attn::BM;
+    kp.num_q_tiles = (r1 + fp8attn::BM - 1) / fp8attn::BM - kp.tile0;
+  }
   kp.scale_log2 = p->scale * fp8attn::LOG2E;
   kp.log2S = (float)std::log2((double)p->S);
   kp.O = p->O;

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_params_layout(lib):
     assert lib.fp8attn_params_sizeof() == ctypes.sizeof(Params)
-    assert lib.fp8attn_version() == 100
+    assert lib.fp8attn_version() == 101
 
 
 def test_status_strings(lib):
@@ -71,6 +71,9 @@ def base_params(**kw):
     (dict(debug_skip_kv_step=-1), EINVAL), (dict(debug_skip_kv_step=2), EINVAL),
     (dict(denominator=2), EINVAL), (dict(denominator=1, S=0.001), EINVAL),
     (dict(qk_dtype=2), EINVAL),
+    (dict(q_begin=64, q_end=256), EINVAL), (dict(q_begin=0, q_end=257), EINVAL),
+    (dict(q_begin=128, q_end=128), EINVAL), (dict(q_begin=-128, q_end=128), EINVAL),
+    (dict(q_begin=0, q_end=200), EINVAL), (dict(q_begin=256, q_end=256), EINVAL),
 ])
 def test_invalid_arguments_rejected_before_launch(lib, kw, status):
     p = base_params(**kw)

@@ -195,6 +195,43 @@ def test_host_tensors_many_chunks(chunks):
     assert torch.equal(st_h.collapse_rows.cpu(), st_d.collapse_rows.cpu())
 
 
+@pytest.mark.parametrize("causal", [0, 1])
+def test_query_row_ranges_compose(causal):
+    """Launches over disjoint query-row ranges (q_begin, q_end), in any order,
+    reproduce one launch over all rows bit for bit, leave the rows outside their
+    range untouched, and their collapse counts add up to the full launch's."""
+    import torch
+    from online_softmax_tcgen05_b200 import O_F32, fp8_attn_fwd_ex
+    B, H, Hkv, N, d = 2, 4, 2, 1000, 128
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 8.0, seed=23)
+    ins = gpu_inputs(W)
+    (Qg, _), (Kg, _), (Vg, _) = ins
+    full, tot, sink_tot, crow = run_gpu(ins, B, H, Hkv, N, d, causal, 256.0, 1, 128, 4)
+    full = full.reshape(B, H, N, d)
+    crow = crow.reshape(B, H, N)
+    dev = Qg.device
+    O = torch.full((B, H, N, d), float("nan"), dtype=torch.float32, device=dev)
+    ctr = torch.zeros(2, dtype=torch.int64, device=dev)
+    rows = torch.full((B, H, N), -1, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    done = np.zeros(N, dtype=bool)
+    for lo, hi in ((384, 640), (896, N), (0, 128), (640, 896), (128, 384)):
+        fp8_attn_fwd_ex(Qg, Kg, Vg, O, B=B, H=H, H_kv=Hkv, N=N, d=d, causal=causal,
+                        scale=1.0 / math.sqrt(d), S=256.0, kv_order=1, n_sink=4, o_dtype=O_F32,
+                        collapse_ctr=ctr[0:1], collapse_sink_ctr=ctr[1:2], collapse_rows=rows,
+                        status_word=status, q_begin=lo, q_end=hi)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, hex(int(status.item()))
+        done[lo:hi] = True
+        Oc, rc = O.cpu().numpy(), rows.cpu().numpy()
+        assert np.array_equal(Oc[:, :, done], full[:, :, done])
+        assert np.isnan(Oc[:, :, ~done]).all()
+        assert np.array_equal(rc[:, :, done], crow[:, :, done])
+        assert (rc[:, :, ~done] == -1).all()
+    c = ctr.cpu().numpy()
+    assert int(c[0]) == tot and int(c[1]) == sink_tot
+
+
 # ------------------------------------------------------------ sweep (cfg 2) --
 @pytest.fixture(scope="module")
 def sweep_inputs():
