@@ -69,6 +69,12 @@ def _launch(q, k, v, o, ctr, rows, *, causal, scale, S, kv_order, n_sink, block_
                     collapse_rows=rows, stream=stream)
 
 
+# Pieces at the start and at the end of the host path that run as one kernel
+# per query head.
+_SPLIT_FIRST = 1
+_SPLIT_LAST = 1
+
+
 def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: float = 256.0,
               kv_order: int = KV_REVERSE, n_sink: int = 0, block_n: int = 0,
               denominator: int = DENOM_FP32_P,
@@ -159,7 +165,8 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
         # compute.  A first or last piece of one kv head therefore runs as one
         # kernel per query head, K and V uploaded once: each head's kernel waits
         # only for its own Q, and each head's O returns as soon as it is done.
-        split = nk == 1 and group > 1 and len(pieces) > 1 and i in (0, len(pieces) - 1)
+        split = (nk == 1 and group > 1 and len(pieces) > 1
+                 and (i < _SPLIT_FIRST or i >= len(pieces) - _SPLIT_LAST))
         subs = [(j, j + 1) for j in range(nq)] if split else [(0, nq)]
         with torch.cuda.stream(pipe.s_in):
             if ev_free is not None:
