@@ -603,9 +603,9 @@ def report_configs(dev):
 
 def report_batched_orders(dev):
     """Batched non-causal configuration (B4 H32 N8192 d128, Delta 10, S 256, counter
-    on): forward and reverse KV order, 3 warm-up pairs then 10 alternating timed
-    pairs (launches 7 and 8 are the first timed forward and reverse ones, for a
-    profiler capture)."""
+    on): forward and reverse KV order, 3 warm-up pairs then 50 alternating timed
+    pairs, median of each (launches 7 and 8 are the first timed forward and
+    reverse ones, for a profiler capture)."""
     import torch
     import workload
     import online_softmax_tcgen05_b200 as fa
@@ -619,7 +619,7 @@ def report_batched_orders(dev):
             r.launch()
     torch.cuda.synchronize()
     times = {name: [] for name, _ in runs}
-    for _ in range(10):
+    for _ in range(50):
         for name, r in runs:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
