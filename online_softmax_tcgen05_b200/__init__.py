@@ -108,6 +108,13 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     kw = dict(causal=causal, scale=scale, S=S, kv_order=kv_order, n_sink=n_sink,
               block_n=block_n, denominator=denominator, o_code=o_code)
     stats = AttentionStats()
+    if B * H * N == 0:   # nothing to compute: an empty O (per-row counts empty too)
+        import torch
+        dev = q.device
+        o = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype, device=dev)
+        if count_collapse and per_row:
+            stats.collapse_rows = torch.zeros((B, H, N), dtype=torch.int32, device=dev)
+        return o, stats
     if q.is_cuda:
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         dev = q.device

@@ -764,7 +764,6 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
     return fail(FP8ATTN_EINVAL, "debug_skip_kv_step needs a status_word to report the timeout");
   if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
     return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
-  if ((long long)p->B * p->H > 65535LL * 65535LL) return fail(FP8ATTN_EINVAL, "B*H too large");
   const bool all_rows = p->q_begin == 0 && p->q_end == 0;
   if (!all_rows) {
     if (p->q_begin < 0 || p->q_end > p->N || p->q_begin >= p->q_end)
@@ -773,6 +772,10 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
       return fail(FP8ATTN_EINVAL, "q_begin must be a multiple of 128, q_end a multiple of 128 or N");
   }
   if ((long long)p->B * p->H * p->N == 0) return FP8ATTN_OK;   // nothing to compute
+  // grid: (query tiles, B*H); causal CTAs are numbered linearly in an int
+  if ((long long)p->B * p->H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
+  if ((long long)((p->N + fp8attn::BM - 1) / fp8attn::BM) * p->B * p->H > 0x7fffffffLL)
+    return fail(FP8ATTN_EINVAL, "too many query tiles: ceil(N / 128) * B * H must be < 2^31");
   if (!p->Q || !p->K || !p->V || !p->O) return fail(FP8ATTN_EINVAL, "Q, K, V, O must be non-NULL");
   if (!aligned16(p->Q) || !aligned16(p->K) || !aligned16(p->V) || !aligned16(p->O))
     return fail(FP8ATTN_EINVAL, "Q, K, V, O must be 16-byte aligned");
@@ -826,7 +829,6 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
   kp.debug_skip_kv_step = p->debug_skip_kv_step;
   kp.denom_cast = p->denominator == FP8ATTN_DENOM_CAST_P;
-  if (kp.B * kp.H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
 
   const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;
   const bool count = p->collapse_ctr != nullptr;

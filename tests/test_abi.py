@@ -74,6 +74,7 @@ def base_params(**kw):
     (dict(q_begin=64, q_end=256), EINVAL), (dict(q_begin=0, q_end=257), EINVAL),
     (dict(q_begin=128, q_end=128), EINVAL), (dict(q_begin=-128, q_end=128), EINVAL),
     (dict(q_begin=0, q_end=200), EINVAL), (dict(q_begin=256, q_end=256), EINVAL),
+    (dict(B=65536, H=1, H_kv=1), EINVAL), (dict(B=256, H=256, H_kv=256), EINVAL),
 ])
 def test_invalid_arguments_rejected_before_launch(lib, kw, status):
     p = base_params(**kw)

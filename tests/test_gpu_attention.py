@@ -195,6 +195,41 @@ def test_host_tensors_many_chunks(chunks):
     assert torch.equal(st_h.collapse_rows.cpu(), st_d.collapse_rows.cpu())
 
 
+def test_empty_problems_are_a_no_op():
+    """B, H or N of zero: the call succeeds, launches nothing and leaves the
+    counters alone; attention() returns an empty O for device and host inputs."""
+    import torch
+    from online_softmax_tcgen05_b200 import attention, fp8_attn_fwd_ex
+    for B, H, Hkv, N in ((0, 2, 1, 128), (1, 0, 0, 128), (1, 2, 1, 0)):
+        q = torch.zeros((B, H, N, 64), dtype=torch.uint8, device="cuda")
+        kv = torch.zeros((B, Hkv, N, 64), dtype=torch.uint8, device="cuda")
+        O = torch.zeros((B, H, N, 64), dtype=torch.bfloat16, device="cuda")
+        ctr = torch.full((2,), 7, dtype=torch.int64, device="cuda")
+        fp8_attn_fwd_ex(q, kv, kv, O, B=B, H=H, H_kv=Hkv, N=N, d=64, causal=1,
+                        collapse_ctr=ctr[0:1], collapse_sink_ctr=ctr[1:2])
+        torch.cuda.synchronize()
+        assert ctr.tolist() == [7, 7]
+        if H > 0:
+            for dev in ("cuda", "cpu"):
+                o, st = attention(q.to(dev), kv.to(dev), kv.to(dev), causal=True,
+                                  count_collapse=True, per_row=True)
+                assert tuple(o.shape) == (B, H, N, 64) and st.collapse == 0
+                assert tuple(st.collapse_rows.shape) == (B, H, N)
+
+
+def test_max_planes_grid():
+    """B * H = 65535 (the largest grid the library accepts) with GQA, a ragged
+    N and 64-key blocks, causal: sampled rows against the oracle, per-row
+    collapse counts exact, first and last planes included."""
+    B, H, Hkv, N, d = 3, 21845, 4369, 65, 64
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 8.0, seed=29)
+    ins = gpu_inputs(W)
+    total = B * H * N
+    rows = sample_rows(B, H, N, 512, seed=3,
+                       include=(0, N - 1, total - N, total - 1, (H - 1) * N + 64))
+    check_case(W, ins, 1, 256.0, 1, 64, rows=rows, what="65535 planes")
+
+
 @pytest.mark.parametrize("causal", [0, 1])
 def test_query_row_ranges_compose(causal):
     """Launches over disjoint query-row ranges (q_begin, q_end), in any order,
