@@ -139,6 +139,7 @@ def fp8_gemm_peak(dev, n=8192, reps=10):
 
 
 KERNEL_SOURCES = ["online_softmax_tcgen05_b200/csrc/fp8_attn_fwd.cu",
+                  "online_softmax_tcgen05_b200/csrc/attn_kernel.cuh",
                   "online_softmax_tcgen05_b200/csrc/sm100.cuh",
                   "online_softmax_tcgen05_b200/csrc/exp2_poly.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_prefill_N32768.json")

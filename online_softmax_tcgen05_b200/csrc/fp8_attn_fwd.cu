@@ -1,6 +1,7 @@
 // fp8_attn_fwd.cu - FP8 (E4M3) attention forward for B200 (sm_100a) with the
-// P-cast scale S and a run-time KV-block order, behind the C ABI of
-// include/fp8attn.h.
+// P-cast scale S and a run-time KV-block order: the kernels and their launch
+// entries (attn_kernel.cuh).  The C ABI of include/fp8attn.h, which validates
+// the arguments and builds the tensor maps, is in fp8attn_abi.cu.
 //
 // Method: "P-Cast Precision in FP8 Attention: Sink-Induced Collapse and the
 // Optimality of S=2^8" (arXiv 2606.06521, gist.science summary).  Section 1
@@ -31,22 +32,17 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <cmath>
 #include <cstdint>
-#include <cstring>
-#include <mutex>
-#include <string>
 
-#include "fp8attn.h"
+#include "attn_kernel.cuh"
 #include "exp2_poly.cuh"
+#include "fp8attn.h"
 #include "sm100.cuh"
 
 namespace fp8attn {
 
-constexpr int BM = 128;         // query rows per CTA (= MMA M, = TMEM lanes)
 constexpr int NSTAGE = 2;       // K/V ring depth
 constexpr int NTHREADS = 192;   // 4 softmax warps + TMA warp + MMA warp
-constexpr float LOG2E = 1.4426950408889634f;
 // Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
 // (exp2_poly.cuh) and the rest on MUFU ex2: the two units then share the
 // exponentials of the softmax.
@@ -54,37 +50,6 @@ constexpr float LOG2E = 1.4426950408889634f;
 #define FP8ATTN_POLY_OF_8 0
 #endif
 constexpr int POLY_OF_8 = FP8ATTN_POLY_OF_8;
-
-// device status codes (status_word): 0x100 | where the wait gave up
-enum : uint32_t {
-  WAIT_PROD_KV_EMPTY = 1,
-  WAIT_MMA_Q = 2,
-  WAIT_MMA_K = 3,
-  WAIT_MMA_S_FREE = 4,
-  WAIT_MMA_V = 5,
-  WAIT_MMA_P = 6,
-  WAIT_SM_S_FULL = 7,
-  WAIT_SM_O_DONE = 8,
-  WAIT_EPI_O_DONE = 9,
-};
-
-struct KParams {
-  int B, H, Hkv, N, group;
-  int causal, kv_order, n_sink;
-  int tile0;          // first query tile of the launch (q_begin / 128)
-  int num_q_tiles;    // query tiles in the launch
-  int sched_group;    // (batch, head) planes per causal scheduling group; divides B * H
-  float scale_log2;   // scale * log2(e)
-  float log2S;   // log2(S): S*p is taken as 2^(s*c - m + log2 S)
-  void* O;
-  unsigned long long* ctr;
-  unsigned long long* ctr_sink;
-  unsigned int* rows;
-  unsigned int* status;
-  unsigned long long timeout_ns;
-  int debug_skip_kv_step;   // testing hook: 1-based KV step whose K load is never issued
-  int denom_cast;           // row sum from the cast values (FP8ATTN_DENOM_CAST_P)
-};
 
 template <int D, int BN, int QB>
 struct Smem {
@@ -616,74 +581,24 @@ __global__ void e4m3_scale_cast_kernel(const float* __restrict__ P, uint8_t* __r
   }
 }
 
-}  // namespace fp8attn
-
-// ======================================================================= host
+// ------------------------------------------------------------- launches --
 namespace {
-
-thread_local std::string g_last_error;
-
-int fail(int status, const std::string& why) {
-  g_last_error = why;
-  return status;
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// 3-D map over a [planes, rows, d] tensor of E4M3 bytes (box [d, box_rows, 1],
-// 128- or 64-byte swizzle by row length) or of BF16 (box [64, box_rows, 1]: one
-// 128-byte swizzle atom per row; a row of d = 128 is loaded as two such panels).
-bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int box_rows,
-              bool bf16) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t esz = bf16 ? 2 : 1;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes};
-  cuuint64_t strides[2] = {(cuuint64_t)d * esz, (cuuint64_t)d * esz * (cuuint64_t)rows};
-  cuuint32_t box[3] = {(cuuint32_t)(bf16 ? 64 : d), (cuuint32_t)box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUtensorMapSwizzle swz = (bf16 || d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B
-                                              : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
-                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int D, int BN, bool OUT_BF16, bool COUNT, int QB>
 cudaError_t launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                   const fp8attn::KParams& kp, cudaStream_t stream) {
-  using L = fp8attn::Smem<D, BN, QB>;
-  auto kern = fp8attn::attn_fwd_kernel<D, BN, OUT_BF16, COUNT, QB>;
+                   const KParams& kp, cudaStream_t stream) {
+  using L = Smem<D, BN, QB>;
+  auto kern = attn_fwd_kernel<D, BN, OUT_BF16, COUNT, QB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(kp.num_q_tiles, kp.B * kp.H);
-  kern<<<grid, fp8attn::NTHREADS, L::ALLOC, stream>>>(q, k, v, kp);
+  kern<<<grid, NTHREADS, L::ALLOC, stream>>>(q, k, v, kp);
   return cudaGetLastError();
 }
 
 template <int D, int BN, int QB>
 cudaError_t launch_q(bool bf16, bool count, const CUtensorMap& q, const CUtensorMap& k,
-                     const CUtensorMap& v, const fp8attn::KParams& kp, cudaStream_t s) {
+                     const CUtensorMap& v, const KParams& kp, cudaStream_t s) {
   if (bf16) return count ? launch<D, BN, true, true, QB>(q, k, v, kp, s)
                          : launch<D, BN, true, false, QB>(q, k, v, kp, s);
   return count ? launch<D, BN, false, true, QB>(q, k, v, kp, s)
@@ -692,7 +607,7 @@ cudaError_t launch_q(bool bf16, bool count, const CUtensorMap& q, const CUtensor
 
 template <int D, int BN>
 cudaError_t launch_dt(bool bf16, bool count, bool qk_bf16, const CUtensorMap& q,
-                      const CUtensorMap& k, const CUtensorMap& v, const fp8attn::KParams& kp,
+                      const CUtensorMap& k, const CUtensorMap& v, const KParams& kp,
                       cudaStream_t s) {
   return qk_bf16 ? launch_q<D, BN, 2>(bf16, count, q, k, v, kp, s)
                  : launch_q<D, BN, 1>(bf16, count, q, k, v, kp, s);
@@ -700,191 +615,24 @@ cudaError_t launch_dt(bool bf16, bool count, bool qk_bf16, const CUtensorMap& q,
 
 }  // namespace
 
-extern "C" {
-
-int fp8attn_version(void) { return 101; }
-
-size_t fp8attn_params_sizeof(void) { return sizeof(fp8attn_params); }
-
-const char* fp8attn_status_string(int status) {
-  switch (status) {
-    case FP8ATTN_OK: return "ok";
-    case FP8ATTN_EINVAL: return "invalid argument";
-    case FP8ATTN_EUNSUPPORTED: return "unsupported configuration";
-    case FP8ATTN_ECUDA: return "CUDA error";
-    case FP8ATTN_ETIMEOUT: return "bounded wait expired on the device";
-    default: return "unknown status";
-  }
+cudaError_t launch_attn(int d, int bn, bool o_bf16, bool count, bool qk_bf16,
+                        const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                        const KParams& kp, cudaStream_t stream) {
+  if (d == 128)
+    return bn == 128 ? launch_dt<128, 128>(o_bf16, count, qk_bf16, q, k, v, kp, stream)
+                     : launch_dt<128, 64>(o_bf16, count, qk_bf16, q, k, v, kp, stream);
+  return bn == 128 ? launch_dt<64, 128>(o_bf16, count, qk_bf16, q, k, v, kp, stream)
+                   : launch_dt<64, 64>(o_bf16, count, qk_bf16, q, k, v, kp, stream);
 }
 
-const char* fp8attn_last_error(void) { return g_last_error.c_str(); }
-
-const char* fp8attn_device_status_string(unsigned int word) {
-  if (word == 0) return "";
-  switch (word & 0xFFu) {
-    case fp8attn::WAIT_PROD_KV_EMPTY: return "timeout: producer waiting for a free K/V stage";
-    case fp8attn::WAIT_MMA_Q: return "timeout: MMA waiting for the Q tile";
-    case fp8attn::WAIT_MMA_K: return "timeout: MMA waiting for a K tile";
-    case fp8attn::WAIT_MMA_S_FREE: return "timeout: MMA waiting for the S buffer";
-    case fp8attn::WAIT_MMA_V: return "timeout: MMA waiting for a V tile";
-    case fp8attn::WAIT_MMA_P: return "timeout: MMA waiting for the P~ tile";
-    case fp8attn::WAIT_SM_S_FULL: return "timeout: softmax waiting for S";
-    case fp8attn::WAIT_SM_O_DONE: return "timeout: softmax waiting for P~V";
-    case fp8attn::WAIT_EPI_O_DONE: return "timeout: epilogue waiting for the last P~V";
-    default: return "timeout: unknown wait";
-  }
-}
-
-int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
-  g_last_error.clear();
-  if (!p) return fail(FP8ATTN_EINVAL, "params is NULL");
-  if (p->B < 0 || p->H < 0 || p->N < 0) return fail(FP8ATTN_EINVAL, "B, H, N must be >= 0");
-  if (p->H_kv <= 0 && p->H > 0) return fail(FP8ATTN_EINVAL, "H_kv must be >= 1");
-  if (p->H > 0 && p->H % p->H_kv) return fail(FP8ATTN_EINVAL, "H must be a multiple of H_kv");
-  if (p->d != 64 && p->d != 128) return fail(FP8ATTN_EUNSUPPORTED, "d must be 64 or 128");
-  const int bn = p->block_n == 0 ? 128 : p->block_n;
-  if (bn != 64 && bn != 128) return fail(FP8ATTN_EUNSUPPORTED, "block_n must be 0, 64 or 128");
-  if (p->causal != 0 && p->causal != 1) return fail(FP8ATTN_EINVAL, "causal must be 0 or 1");
-  if (!std::isfinite(p->scale) || !(p->scale > 0.f))
-    return fail(FP8ATTN_EINVAL, "scale must be finite and > 0");
-  if (!std::isfinite(p->S) || !(p->S > 0.f)) return fail(FP8ATTN_EINVAL, "S must be finite and > 0");
-  if (p->kv_order != FP8ATTN_KV_FORWARD && p->kv_order != FP8ATTN_KV_REVERSE)
-    return fail(FP8ATTN_EINVAL, "kv_order must be 0 (forward) or 1 (reverse)");
-  if (p->n_sink < 0 || p->n_sink > p->N) return fail(FP8ATTN_EINVAL, "n_sink must be in [0, N]");
-  if (p->denominator != FP8ATTN_DENOM_FP32_P && p->denominator != FP8ATTN_DENOM_CAST_P)
-    return fail(FP8ATTN_EINVAL, "denominator must be FP8ATTN_DENOM_FP32_P or FP8ATTN_DENOM_CAST_P");
-  if (p->denominator == FP8ATTN_DENOM_CAST_P && std::isfinite(p->S) && p->S < 0x1p-8f)
-    return fail(FP8ATTN_EINVAL, "the cast-value denominator needs S >= 2^-8");
-  if (p->qk_dtype != FP8ATTN_QK_E4M3 && p->qk_dtype != FP8ATTN_QK_BF16)
-    return fail(FP8ATTN_EINVAL, "qk_dtype must be FP8ATTN_QK_E4M3 or FP8ATTN_QK_BF16");
-  if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
-    return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
-  if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
-  if (p->debug_skip_kv_step > 0 && !p->status_word)
-    return fail(FP8ATTN_EINVAL, "debug_skip_kv_step needs a status_word to report the timeout");
-  if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
-    return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
-  const bool all_rows = p->q_begin == 0 && p->q_end == 0;
-  if (!all_rows) {
-    if (p->q_begin < 0 || p->q_end > p->N || p->q_begin >= p->q_end)
-      return fail(FP8ATTN_EINVAL, "q_begin, q_end must satisfy 0 <= q_begin < q_end <= N");
-    if (p->q_begin % fp8attn::BM || (p->q_end % fp8attn::BM && p->q_end != p->N))
-      return fail(FP8ATTN_EINVAL, "q_begin must be a multiple of 128, q_end a multiple of 128 or N");
-  }
-  if ((long long)p->B * p->H * p->N == 0) return FP8ATTN_OK;   // nothing to compute
-  // grid: (query tiles, B*H); causal CTAs are numbered linearly in an int
-  if ((long long)p->B * p->H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
-  if ((long long)((p->N + fp8attn::BM - 1) / fp8attn::BM) * p->B * p->H > 0x7fffffffLL)
-    return fail(FP8ATTN_EINVAL, "too many query tiles: ceil(N / 128) * B * H must be < 2^31");
-  if (!p->Q || !p->K || !p->V || !p->O) return fail(FP8ATTN_EINVAL, "Q, K, V, O must be non-NULL");
-  if (!aligned16(p->Q) || !aligned16(p->K) || !aligned16(p->V) || !aligned16(p->O))
-    return fail(FP8ATTN_EINVAL, "Q, K, V, O must be 16-byte aligned");
-  if ((p->collapse_ctr && ((uintptr_t)p->collapse_ctr & 7)) ||
-      (p->collapse_sink_ctr && ((uintptr_t)p->collapse_sink_ctr & 7)) ||
-      (p->collapse_rows && ((uintptr_t)p->collapse_rows & 3)) ||
-      (p->status_word && ((uintptr_t)p->status_word & 3)))
-    return fail(FP8ATTN_EINVAL, "counter / status pointers must be naturally aligned");
-
-  CUtensorMap mq, mk, mv;
-  if (!encode_fn()) return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled is not available");
-  const bool qkb = p->qk_dtype == FP8ATTN_QK_BF16;
-  if (!make_map(&mq, p->Q, p->d, p->N, p->B * p->H, fp8attn::BM, qkb) ||
-      !make_map(&mk, p->K, p->d, p->N, p->B * p->H_kv, bn, qkb) ||
-      !make_map(&mv, p->V, p->d, p->N, p->B * p->H_kv, bn, false))
-    return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled failed");
-
-  fp8attn::KParams kp;
-  kp.B = p->B;
-  kp.H = p->H;
-  kp.Hkv = p->H_kv;
-  kp.N = p->N;
-  kp.group = p->H / p->H_kv;
-  {
-    // scheduling group: the query heads of as many KV heads as keep their K and V
-    // (N * d bytes each, K in BF16 takes twice that) within 32 MiB, a quarter of
-    // the L2 (measured: half the L2 lost 0.4% at N = 131072, where a group is one
-    // KV head; the whole problem at once lost 4% there)
-    const double kv_bytes = (double)p->N * p->d * (p->qk_dtype == FP8ATTN_QK_BF16 ? 3.0 : 2.0);
-    const int nkv = p->B * p->H_kv;
-    int kvg = (int)(32.0 * 1024.0 * 1024.0 / kv_bytes);
-    kvg = kvg < 1 ? 1 : (kvg > nkv ? nkv : kvg);
-    while (nkv % kvg) --kvg;
-    kp.sched_group = kvg * kp.group;
-  }
-  kp.causal = p->causal;
-  kp.kv_order = p->kv_order;
-  kp.n_sink = p->n_sink;
-  {
-    const int r0 = all_rows ? 0 : p->q_begin, r1 = all_rows ? p->N : p->q_end;
-    kp.tile0 = r0 / fp8attn::BM;
-    kp.num_q_tiles = (r1 + fp8attn::BM - 1) / fp8attn::BM - kp.tile0;
-  }
-  kp.scale_log2 = p->scale * fp8attn::LOG2E;
-  kp.log2S = (float)std::log2((double)p->S);
-  kp.O = p->O;
-  kp.ctr = p->collapse_ctr;
-  kp.ctr_sink = p->collapse_sink_ctr;
-  kp.rows = p->collapse_rows;
-  kp.status = p->status_word;
-  kp.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
-  kp.debug_skip_kv_step = p->debug_skip_kv_step;
-  kp.denom_cast = p->denominator == FP8ATTN_DENOM_CAST_P;
-
-  const bool bf16 = p->o_dtype == FP8ATTN_O_BF16;
-  const bool count = p->collapse_ctr != nullptr;
-  const bool qk_bf16 = p->qk_dtype == FP8ATTN_QK_BF16;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (p->d == 128)
-    e = (bn == 128) ? launch_dt<128, 128>(bf16, count, qk_bf16, mq, mk, mv, kp, s)
-                    : launch_dt<128, 64>(bf16, count, qk_bf16, mq, mk, mv, kp, s);
-  else
-    e = (bn == 128) ? launch_dt<64, 128>(bf16, count, qk_bf16, mq, mk, mv, kp, s)
-                    : launch_dt<64, 64>(bf16, count, qk_bf16, mq, mk, mv, kp, s);
-  if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
-  return FP8ATTN_OK;
-}
-
-int fp8_attn_fwd(const void* Q, const void* K, const void* V, void* O, int B, int H, int N, int d,
-                 int causal, float scale, float S, int kv_order, int n_sink,
-                 unsigned long long* collapse_ctr, fp8attn_stream_t stream) {
-  fp8attn_params p;
-  std::memset(&p, 0, sizeof(p));
-  p.Q = Q;
-  p.K = K;
-  p.V = V;
-  p.O = O;
-  p.B = B;
-  p.H = H;
-  p.H_kv = H;
-  p.N = N;
-  p.d = d;
-  p.causal = causal;
-  p.scale = scale;
-  p.S = S;
-  p.kv_order = kv_order;
-  p.n_sink = n_sink;
-  p.o_dtype = FP8ATTN_O_BF16;
-  p.block_n = 128;
-  p.collapse_ctr = collapse_ctr;
-  return fp8_attn_fwd_ex(&p, stream);
-}
-
-int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
-                        fp8attn_stream_t stream) {
-  g_last_error.clear();
-  if (n == 0) return FP8ATTN_OK;
-  if (!P || !out) return fail(FP8ATTN_EINVAL, "P and out must be non-NULL");
-  if (!aligned16(P) || !aligned16(out)) return fail(FP8ATTN_EINVAL, "P and out must be 16-byte aligned");
-  if (!std::isfinite(S)) return fail(FP8ATTN_EINVAL, "S must be finite");
+cudaError_t launch_e4m3_scale_cast(const float* P, uint8_t* out, size_t n, float S,
+                                   cudaStream_t stream) {
   const size_t n8 = n / 8;
-  int blocks = (int)std::min<size_t>((n8 + 255) / 256, (size_t)148 * 16);
+  size_t blocks = (n8 + 255) / 256;
+  if (blocks > (size_t)148 * 16) blocks = (size_t)148 * 16;
   if (blocks < 1) blocks = 1;
-  fp8attn::e4m3_scale_cast_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      P, out, n, S);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
-  return FP8ATTN_OK;
+  e4m3_scale_cast_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P, out, n, S);
+  return cudaGetLastError();
 }
 
-}  // extern "C"
+}  // namespace fp8attn
