@@ -26,8 +26,9 @@
  * Causal: key j is visible to query i iff j <= i (square prefill, no offset).
  *
  * Conventions for every entry point:
- *   - Tensor pointers are DEVICE pointers owned by the caller.  The library
- *     never frees or retains them and allocates no device memory.
+ *   - Tensor pointers are DEVICE pointers owned by the caller (except Q, K, V, O
+ *     of fp8_attn_fwd_host, which are host memory).  The library never frees or
+ *     retains them and allocates no device memory.
  *   - All work is enqueued asynchronously on `stream` (NULL = legacy default
  *     stream).  A return of FP8ATTN_OK means "validated and launched".
  *   - Arguments are validated on the host before anything is launched; an
@@ -140,6 +141,50 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream);
  * both 16-byte aligned.  S finite (any sign).  NaN -> 0x7F, |x| > 448 -> +-448. */
 int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
                         fp8attn_stream_t stream);
+
+/* ---------------------------------------------------- host-buffer entry ---
+ * fp8_attn_fwd_host - the same operation for Q, K, V and O in HOST memory:
+ * the copies to and from the device run inside the call's stream work,
+ * pipelined against the kernels.
+ *
+ * The problem is cut into up to host_chunks pieces of whole (batch, kv-head)
+ * units, none crossing a batch element.  Each piece's K and V (and Q, per
+ * sub-step) are copied into one of three staging sets in `workspace`, its
+ * kernels run on two compute streams taken in turn, and each sub-step's O is
+ * copied back as soon as its kernel is done.  The first and last pieces, when
+ * they hold one kv head of several query heads, run one kernel per query head.
+ *
+ *   p            as for fp8_attn_fwd_ex, but Q, K, V, O are HOST pointers:
+ *                page-locked memory lets the copies overlap the kernels
+ *                (pageable memory works, with the copies serialised).
+ *                collapse_ctr, collapse_sink_ctr, collapse_rows and status_word
+ *                stay DEVICE pointers.  q_begin = q_end = 0 (all rows).
+ *   plan         from fp8attn_host_plan_create on the current device.
+ *   workspace    DEVICE memory, 256-byte aligned, of at least
+ *                fp8attn_host_workspace_bytes(p, host_chunks) bytes, owned by
+ *                the caller; not to be reused before `stream` has passed this call.
+ *   host_chunks  >= 1; the number of pieces (at most B * H_kv).
+ *   stream       the work starts after prior work on `stream`, and `stream` is
+ *                ordered after the last copy back: synchronise it before reading
+ *                O or the counters.
+ * Returns an fp8attn_status.  A failure after work was enqueued (FP8ATTN_ECUDA)
+ * leaves O incomplete and the plan's streams possibly busy. */
+typedef struct fp8attn_host_plan fp8attn_host_plan;   /* opaque */
+
+/* Streams and events of the host pipeline, on the current device.  A plan
+ * serves one call at a time (not for concurrent use from several threads) and
+ * may be reused by any number of calls. */
+int fp8attn_host_plan_create(fp8attn_host_plan** plan);
+
+/* Waits for the plan's streams, then releases them.  NULL is a no-op. */
+int fp8attn_host_plan_destroy(fp8attn_host_plan* plan);
+
+/* Device workspace bytes that fp8_attn_fwd_host needs for p and host_chunks
+ * (0 for an empty or invalid shape). */
+size_t fp8attn_host_workspace_bytes(const fp8attn_params* p, int host_chunks);
+
+int fp8_attn_fwd_host(const fp8attn_params* p, fp8attn_host_plan* plan, void* workspace,
+                      size_t workspace_bytes, int host_chunks, fp8attn_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* fp8attn_status_string(int status);

@@ -53,6 +53,11 @@ SIGNATURES = {
     "fp8attn_device_status_string": ([ctypes.c_uint], ctypes.c_char_p),
     "fp8attn_version": ([], ctypes.c_int),
     "fp8attn_params_sizeof": ([], ctypes.c_size_t),
+    "fp8attn_host_plan_create": ([ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+    "fp8attn_host_plan_destroy": ([ctypes.c_void_p], ctypes.c_int),
+    "fp8attn_host_workspace_bytes": ([ctypes.POINTER(Params), ctypes.c_int], ctypes.c_size_t),
+    "fp8_attn_fwd_host": ([ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_void_p,
+                           ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
 }
 
 _lib = None
@@ -121,24 +126,73 @@ def fp8_attn_fwd(Q, K, V, O, B, H, N, d, causal, scale, S, kv_order, n_sink, col
            "fp8_attn_fwd")
 
 
-def fp8_attn_fwd_ex(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S=256.0,
-                    kv_order=KV_REVERSE, n_sink=0, o_dtype=O_BF16, block_n=0, denominator=0,
-                    qk_dtype=QK_E4M3,
-                    collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None,
-                    status_word=None, timeout_ns=0, debug_skip_kv_step=0, q_begin=0, q_end=0,
-                    stream=None):
-    """Full-parameter entry point (all tensors on the device).  ``q_begin``,
-    ``q_end``: the query-row range of each (batch, head) plane to compute
-    (0, 0 = all rows)."""
-    p = Params(Q=Q.data_ptr(), K=K.data_ptr(), V=V.data_ptr(), O=O.data_ptr(),
-               B=B, H=H, H_kv=H_kv, N=N, d=d, causal=int(causal),
-               scale=float(scale if scale is not None else 1.0 / math.sqrt(d)), S=float(S),
-               kv_order=int(kv_order), n_sink=int(n_sink), o_dtype=int(o_dtype),
-               block_n=int(block_n), denominator=int(denominator), qk_dtype=int(qk_dtype),
-               collapse_ctr=None if collapse_ctr is None else collapse_ctr.data_ptr(),
-               collapse_sink_ctr=None if collapse_sink_ctr is None else collapse_sink_ctr.data_ptr(),
-               collapse_rows=None if collapse_rows is None else collapse_rows.data_ptr(),
-               status_word=None if status_word is None else status_word.data_ptr(),
-               timeout_ns=int(timeout_ns), debug_skip_kv_step=int(debug_skip_kv_step),
-               q_begin=int(q_begin), q_end=int(q_end))
+def _params(Q, K, V, O, *, B, H, H_kv, N, d, causal=False, scale=None, S=256.0,
+            kv_order=KV_REVERSE, n_sink=0, o_dtype=O_BF16, block_n=0, denominator=0,
+            qk_dtype=QK_E4M3, collapse_ctr=None, collapse_sink_ctr=None, collapse_rows=None,
+            status_word=None, timeout_ns=0, debug_skip_kv_step=0, q_begin=0, q_end=0):
+    return Params(Q=Q.data_ptr(), K=K.data_ptr(), V=V.data_ptr(), O=O.data_ptr(),
+                  B=B, H=H, H_kv=H_kv, N=N, d=d, causal=int(causal),
+                  scale=float(scale if scale is not None else 1.0 / math.sqrt(d)), S=float(S),
+                  kv_order=int(kv_order), n_sink=int(n_sink), o_dtype=int(o_dtype),
+                  block_n=int(block_n), denominator=int(denominator), qk_dtype=int(qk_dtype),
+                  collapse_ctr=None if collapse_ctr is None else collapse_ctr.data_ptr(),
+                  collapse_sink_ctr=(None if collapse_sink_ctr is None
+                                     else collapse_sink_ctr.data_ptr()),
+                  collapse_rows=None if collapse_rows is None else collapse_rows.data_ptr(),
+                  status_word=None if status_word is None else status_word.data_ptr(),
+                  timeout_ns=int(timeout_ns), debug_skip_kv_step=int(debug_skip_kv_step),
+                  q_begin=int(q_begin), q_end=int(q_end))
+
+
+def fp8_attn_fwd_ex(Q, K, V, O, *, stream=None, **kw):
+    """Full-parameter entry point (all tensors on the device).  Keywords are the
+    fields of fp8attn_params (B, H, H_kv, N, d required); ``q_begin``, ``q_end``:
+    the query-row range of each (batch, head) plane to compute (0, 0 = all rows)."""
+    p = _params(Q, K, V, O, **kw)
     _check(load_library().fp8_attn_fwd_ex(ctypes.byref(p), _stream(stream)), "fp8_attn_fwd_ex")
+
+
+class HostPlan:
+    """The streams and events of the host-buffer pipeline (fp8attn_host_plan),
+    created on the current device; reusable across calls, one call at a time."""
+
+    def __init__(self):
+        h = ctypes.c_void_p()
+        _check(load_library().fp8attn_host_plan_create(ctypes.byref(h)),
+               "fp8attn_host_plan_create")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            load_library().fp8attn_host_plan_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def host_workspace_bytes(*, B, H, H_kv, N, d, qk_dtype=QK_E4M3, o_dtype=O_BF16,
+                         host_chunks=16) -> int:
+    """Device workspace bytes that fp8_attn_fwd_host needs for this shape."""
+    p = Params(B=B, H=H, H_kv=H_kv, N=N, d=d, qk_dtype=int(qk_dtype), o_dtype=int(o_dtype))
+    return int(load_library().fp8attn_host_workspace_bytes(ctypes.byref(p), int(host_chunks)))
+
+
+def fp8_attn_fwd_host(Q, K, V, O, *, plan, workspace, host_chunks=16, stream=None, **kw):
+    """Host-buffer entry point: Q, K, V, O are CPU tensors (pinned for overlap),
+    counters and per-row counts CUDA tensors, ``workspace`` a CUDA byte tensor of
+    at least host_workspace_bytes(...) bytes.  Ordered after prior work on
+    ``stream`` (default: current); synchronise it before reading O."""
+    p = _params(Q, K, V, O, **kw)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load_library().fp8_attn_fwd_host(ctypes.byref(p), plan.handle,
+                                            ctypes.c_void_p(workspace.data_ptr()), nbytes,
+                                            int(host_chunks), _stream(stream)),
+           "fp8_attn_fwd_host")

@@ -11,17 +11,85 @@
 #include <mutex>
 #include <string>
 
+#include "abi_internal.h"
 #include "attn_kernel.cuh"
 #include "fp8attn.h"
 
-namespace {
+namespace fp8attn {
 
+namespace {
 thread_local std::string g_last_error;
+}  // namespace
 
 int fail(int status, const std::string& why) {
   g_last_error = why;
   return status;
 }
+
+void clear_error() { g_last_error.clear(); }
+
+const char* last_error() { return g_last_error.c_str(); }
+
+int validate(const fp8attn_params* p, bool host_buffers) {
+  if (!p) return fail(FP8ATTN_EINVAL, "params is NULL");
+  if (p->B < 0 || p->H < 0 || p->N < 0) return fail(FP8ATTN_EINVAL, "B, H, N must be >= 0");
+  if (p->H_kv <= 0 && p->H > 0) return fail(FP8ATTN_EINVAL, "H_kv must be >= 1");
+  if (p->H > 0 && p->H % p->H_kv) return fail(FP8ATTN_EINVAL, "H must be a multiple of H_kv");
+  if (p->d != 64 && p->d != 128) return fail(FP8ATTN_EUNSUPPORTED, "d must be 64 or 128");
+  const int bn = p->block_n == 0 ? 128 : p->block_n;
+  if (bn != 64 && bn != 128) return fail(FP8ATTN_EUNSUPPORTED, "block_n must be 0, 64 or 128");
+  if (p->causal != 0 && p->causal != 1) return fail(FP8ATTN_EINVAL, "causal must be 0 or 1");
+  if (!std::isfinite(p->scale) || !(p->scale > 0.f))
+    return fail(FP8ATTN_EINVAL, "scale must be finite and > 0");
+  if (!std::isfinite(p->S) || !(p->S > 0.f)) return fail(FP8ATTN_EINVAL, "S must be finite and > 0");
+  if (p->kv_order != FP8ATTN_KV_FORWARD && p->kv_order != FP8ATTN_KV_REVERSE)
+    return fail(FP8ATTN_EINVAL, "kv_order must be 0 (forward) or 1 (reverse)");
+  if (p->n_sink < 0 || p->n_sink > p->N) return fail(FP8ATTN_EINVAL, "n_sink must be in [0, N]");
+  if (p->denominator != FP8ATTN_DENOM_FP32_P && p->denominator != FP8ATTN_DENOM_CAST_P)
+    return fail(FP8ATTN_EINVAL, "denominator must be FP8ATTN_DENOM_FP32_P or FP8ATTN_DENOM_CAST_P");
+  if (p->denominator == FP8ATTN_DENOM_CAST_P && std::isfinite(p->S) && p->S < 0x1p-8f)
+    return fail(FP8ATTN_EINVAL, "the cast-value denominator needs S >= 2^-8");
+  if (p->qk_dtype != FP8ATTN_QK_E4M3 && p->qk_dtype != FP8ATTN_QK_BF16)
+    return fail(FP8ATTN_EINVAL, "qk_dtype must be FP8ATTN_QK_E4M3 or FP8ATTN_QK_BF16");
+  if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
+    return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
+  if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
+  if (p->debug_skip_kv_step > 0 && !p->status_word)
+    return fail(FP8ATTN_EINVAL, "debug_skip_kv_step needs a status_word to report the timeout");
+  if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
+    return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
+  const bool all_rows = p->q_begin == 0 && p->q_end == 0;
+  if (!all_rows) {
+    if (host_buffers)
+      return fail(FP8ATTN_EINVAL, "the host-buffer entry computes all rows: q_begin = q_end = 0");
+    if (p->q_begin < 0 || p->q_end > p->N || p->q_begin >= p->q_end)
+      return fail(FP8ATTN_EINVAL, "q_begin, q_end must satisfy 0 <= q_begin < q_end <= N");
+    if (p->q_begin % BM || (p->q_end % BM && p->q_end != p->N))
+      return fail(FP8ATTN_EINVAL, "q_begin must be a multiple of 128, q_end a multiple of 128 or N");
+  }
+  if ((long long)p->B * p->H * p->N == 0) return 1;   // nothing to compute
+  // grid: (query tiles, B*H); causal CTAs are numbered linearly in an int
+  if ((long long)p->B * p->H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
+  if ((long long)((p->N + BM - 1) / BM) * p->B * p->H > 0x7fffffffLL)
+    return fail(FP8ATTN_EINVAL, "too many query tiles: ceil(N / 128) * B * H must be < 2^31");
+  if (!p->Q || !p->K || !p->V || !p->O) return fail(FP8ATTN_EINVAL, "Q, K, V, O must be non-NULL");
+  if (!host_buffers && (!aligned16(p->Q) || !aligned16(p->K) || !aligned16(p->V) ||
+                        !aligned16(p->O)))
+    return fail(FP8ATTN_EINVAL, "Q, K, V, O must be 16-byte aligned");
+  if ((p->collapse_ctr && ((uintptr_t)p->collapse_ctr & 7)) ||
+      (p->collapse_sink_ctr && ((uintptr_t)p->collapse_sink_ctr & 7)) ||
+      (p->collapse_rows && ((uintptr_t)p->collapse_rows & 3)) ||
+      (p->status_word && ((uintptr_t)p->status_word & 3)))
+    return fail(FP8ATTN_EINVAL, "counter / status pointers must be naturally aligned");
+  return 0;
+}
+
+}  // namespace fp8attn
+
+namespace {
+
+using fp8attn::aligned16;
+using fp8attn::fail;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -62,7 +130,6 @@ bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int
   return r == CUDA_SUCCESS;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -83,7 +150,7 @@ const char* fp8attn_status_string(int status) {
   }
 }
 
-const char* fp8attn_last_error(void) { return g_last_error.c_str(); }
+const char* fp8attn_last_error(void) { return fp8attn::last_error(); }
 
 const char* fp8attn_device_status_string(unsigned int word) {
   if (word == 0) return "";
@@ -102,54 +169,11 @@ const char* fp8attn_device_status_string(unsigned int word) {
 }
 
 int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
-  g_last_error.clear();
-  if (!p) return fail(FP8ATTN_EINVAL, "params is NULL");
-  if (p->B < 0 || p->H < 0 || p->N < 0) return fail(FP8ATTN_EINVAL, "B, H, N must be >= 0");
-  if (p->H_kv <= 0 && p->H > 0) return fail(FP8ATTN_EINVAL, "H_kv must be >= 1");
-  if (p->H > 0 && p->H % p->H_kv) return fail(FP8ATTN_EINVAL, "H must be a multiple of H_kv");
-  if (p->d != 64 && p->d != 128) return fail(FP8ATTN_EUNSUPPORTED, "d must be 64 or 128");
+  fp8attn::clear_error();
+  const int v = fp8attn::validate(p, false);
+  if (v < 0) return v;
+  if (v == 1) return FP8ATTN_OK;   // nothing to compute
   const int bn = p->block_n == 0 ? 128 : p->block_n;
-  if (bn != 64 && bn != 128) return fail(FP8ATTN_EUNSUPPORTED, "block_n must be 0, 64 or 128");
-  if (p->causal != 0 && p->causal != 1) return fail(FP8ATTN_EINVAL, "causal must be 0 or 1");
-  if (!std::isfinite(p->scale) || !(p->scale > 0.f))
-    return fail(FP8ATTN_EINVAL, "scale must be finite and > 0");
-  if (!std::isfinite(p->S) || !(p->S > 0.f)) return fail(FP8ATTN_EINVAL, "S must be finite and > 0");
-  if (p->kv_order != FP8ATTN_KV_FORWARD && p->kv_order != FP8ATTN_KV_REVERSE)
-    return fail(FP8ATTN_EINVAL, "kv_order must be 0 (forward) or 1 (reverse)");
-  if (p->n_sink < 0 || p->n_sink > p->N) return fail(FP8ATTN_EINVAL, "n_sink must be in [0, N]");
-  if (p->denominator != FP8ATTN_DENOM_FP32_P && p->denominator != FP8ATTN_DENOM_CAST_P)
-    return fail(FP8ATTN_EINVAL, "denominator must be FP8ATTN_DENOM_FP32_P or FP8ATTN_DENOM_CAST_P");
-  if (p->denominator == FP8ATTN_DENOM_CAST_P && std::isfinite(p->S) && p->S < 0x1p-8f)
-    return fail(FP8ATTN_EINVAL, "the cast-value denominator needs S >= 2^-8");
-  if (p->qk_dtype != FP8ATTN_QK_E4M3 && p->qk_dtype != FP8ATTN_QK_BF16)
-    return fail(FP8ATTN_EINVAL, "qk_dtype must be FP8ATTN_QK_E4M3 or FP8ATTN_QK_BF16");
-  if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
-    return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
-  if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
-  if (p->debug_skip_kv_step > 0 && !p->status_word)
-    return fail(FP8ATTN_EINVAL, "debug_skip_kv_step needs a status_word to report the timeout");
-  if ((p->collapse_sink_ctr || p->collapse_rows) && !p->collapse_ctr)
-    return fail(FP8ATTN_EINVAL, "collapse_sink_ctr / collapse_rows need collapse_ctr");
-  const bool all_rows = p->q_begin == 0 && p->q_end == 0;
-  if (!all_rows) {
-    if (p->q_begin < 0 || p->q_end > p->N || p->q_begin >= p->q_end)
-      return fail(FP8ATTN_EINVAL, "q_begin, q_end must satisfy 0 <= q_begin < q_end <= N");
-    if (p->q_begin % fp8attn::BM || (p->q_end % fp8attn::BM && p->q_end != p->N))
-      return fail(FP8ATTN_EINVAL, "q_begin must be a multiple of 128, q_end a multiple of 128 or N");
-  }
-  if ((long long)p->B * p->H * p->N == 0) return FP8ATTN_OK;   // nothing to compute
-  // grid: (query tiles, B*H); causal CTAs are numbered linearly in an int
-  if ((long long)p->B * p->H > 65535) return fail(FP8ATTN_EINVAL, "B*H must be <= 65535");
-  if ((long long)((p->N + fp8attn::BM - 1) / fp8attn::BM) * p->B * p->H > 0x7fffffffLL)
-    return fail(FP8ATTN_EINVAL, "too many query tiles: ceil(N / 128) * B * H must be < 2^31");
-  if (!p->Q || !p->K || !p->V || !p->O) return fail(FP8ATTN_EINVAL, "Q, K, V, O must be non-NULL");
-  if (!aligned16(p->Q) || !aligned16(p->K) || !aligned16(p->V) || !aligned16(p->O))
-    return fail(FP8ATTN_EINVAL, "Q, K, V, O must be 16-byte aligned");
-  if ((p->collapse_ctr && ((uintptr_t)p->collapse_ctr & 7)) ||
-      (p->collapse_sink_ctr && ((uintptr_t)p->collapse_sink_ctr & 7)) ||
-      (p->collapse_rows && ((uintptr_t)p->collapse_rows & 3)) ||
-      (p->status_word && ((uintptr_t)p->status_word & 3)))
-    return fail(FP8ATTN_EINVAL, "counter / status pointers must be naturally aligned");
 
   CUtensorMap mq, mk, mv;
   if (!encode_fn()) return fail(FP8ATTN_ECUDA, "cuTensorMapEncodeTiled is not available");
@@ -181,6 +205,7 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   kp.kv_order = p->kv_order;
   kp.n_sink = p->n_sink;
   {
+    const bool all_rows = p->q_begin == 0 && p->q_end == 0;
     const int r0 = all_rows ? 0 : p->q_begin, r1 = all_rows ? p->N : p->q_end;
     kp.tile0 = r0 / fp8attn::BM;
     kp.num_q_tiles = (r1 + fp8attn::BM - 1) / fp8attn::BM - kp.tile0;
@@ -232,7 +257,7 @@ int fp8_attn_fwd(const void* Q, const void* K, const void* V, void* O, int B, in
 
 int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
                         fp8attn_stream_t stream) {
-  g_last_error.clear();
+  fp8attn::clear_error();
   if (n == 0) return FP8ATTN_OK;
   if (!P || !out) return fail(FP8ATTN_EINVAL, "P and out must be non-NULL");
   if (!aligned16(P) || !aligned16(out)) return fail(FP8ATTN_EINVAL, "P and out must be 16-byte aligned");

@@ -101,3 +101,42 @@ def test_cast_validation(lib):
     assert lib.fp8_e4m3_scale_cast(None, FAKE, 16, 1.0, None) == EINVAL
     assert lib.fp8_e4m3_scale_cast(FAKE, FAKE, 16, float("nan"), None) == EINVAL
     assert lib.fp8_e4m3_scale_cast(FAKE + 4, FAKE, 16, 1.0, None) == EINVAL
+
+
+# ------------------------------------------------- host-buffer entry (no GPU) --
+def test_host_workspace_bytes(lib):
+    # prefill, 16 chunks -> 8 pieces of one kv head: 3 sets of Q (4 heads), K, V, O (BF16)
+    plane = 32768 * 128
+    assert _binding.host_workspace_bytes(B=1, H=32, H_kv=8, N=32768, d=128) == \
+        3 * (4 * plane + plane + plane + 4 * plane * 2)
+    # one chunk: the whole problem is one piece
+    assert _binding.host_workspace_bytes(B=1, H=32, H_kv=8, N=32768, d=128, host_chunks=1) == \
+        3 * 8 * (4 * plane + plane + plane + 4 * plane * 2)
+    # BF16 Q/K, FP32 O, sizes rounded up to 256 bytes
+    n, d = 100, 64
+    r = lambda x: (x + 255) // 256 * 256
+    assert _binding.host_workspace_bytes(B=2, H=4, H_kv=2, N=n, d=d, qk_dtype=1, o_dtype=1,
+                                         host_chunks=4) == \
+        3 * (r(2 * n * d * 2) + r(n * d * 2) + r(n * d) + r(2 * n * d * 4))
+    for bad in (dict(B=0), dict(N=0), dict(H=3), dict(H_kv=0)):
+        kw = dict(B=1, H=4, H_kv=2, N=256, d=64)
+        kw.update(bad)
+        assert _binding.host_workspace_bytes(**kw) == 0
+    assert _binding.host_workspace_bytes(B=1, H=4, H_kv=2, N=256, d=64, host_chunks=0) == 0
+
+
+@pytest.mark.parametrize("kw,plan,ws,nbytes,chunks", [
+    (dict(q_begin=128, q_end=256), FAKE, 0x100000, 1 << 40, 4),   # row ranges: device entry only
+    (dict(d=96), FAKE, 0x100000, 1 << 40, 4),
+    (dict(), None, 0x100000, 1 << 40, 4),                          # no plan
+    (dict(), FAKE, 0x100000, 1 << 40, 0),                          # host_chunks < 1
+    (dict(), FAKE, None, 1 << 40, 4),                              # no workspace
+    (dict(), FAKE, 0x100080, 1 << 40, 4),                          # workspace not 256-aligned
+    (dict(), FAKE, 0x100000, 1024, 4),                             # workspace too small
+    (dict(Q=None), FAKE, 0x100000, 1 << 40, 4),
+])
+def test_host_entry_rejects_before_any_cuda_call(lib, kw, plan, ws, nbytes, chunks):
+    p = base_params(**kw)
+    st = lib.fp8_attn_fwd_host(ctypes.byref(p), plan, ws, nbytes, chunks, None)
+    assert st in (EINVAL, EUNSUPPORTED)
+    assert _binding.last_error() != ""

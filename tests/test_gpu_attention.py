@@ -195,6 +195,59 @@ def test_host_tensors_many_chunks(chunks):
     assert torch.equal(st_h.collapse_rows.cpu(), st_d.collapse_rows.cpu())
 
 
+@pytest.mark.parametrize("qk_bf16,o_f32,pinned", [(False, False, True), (True, True, False)])
+def test_host_entry_direct(qk_bf16, o_f32, pinned):
+    """fp8_attn_fwd_host called directly on a side stream, twice with one plan and
+    workspace (the second call reuses every staging set): O, the counters and the
+    per-row counts equal the device entry's bit for bit, with pinned or pageable
+    host memory, E4M3 or BF16 Q/K, BF16 or FP32 O."""
+    import torch
+    from online_softmax_tcgen05_b200 import (O_BF16, O_F32, QK_BF16, QK_E4M3, HostPlan,
+                                             fp8_attn_fwd_ex, fp8_attn_fwd_host,
+                                             host_workspace_bytes)
+    B, H, Hkv, N, d = 2, 6, 3, 700, 128
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 8.0, seed=31)
+    if qk_bf16:
+        ins = gpu_inputs_bf16(W)
+    else:
+        ins = gpu_inputs(W)
+    (Qg, _), (Kg, _), (Vg, _) = ins
+    o_dt = torch.float32 if o_f32 else torch.bfloat16
+    kw = dict(B=B, H=H, H_kv=Hkv, N=N, d=d, causal=1, S=256.0, kv_order=1, n_sink=4,
+              o_dtype=O_F32 if o_f32 else O_BF16, qk_dtype=QK_BF16 if qk_bf16 else QK_E4M3)
+    dev = Qg.device
+    Od = torch.empty((B, H, N, d), dtype=o_dt, device=dev)
+    ctr_d = torch.zeros(2, dtype=torch.int64, device=dev)
+    rows_d = torch.zeros((B, H, N), dtype=torch.int32, device=dev)
+    fp8_attn_fwd_ex(Qg, Kg, Vg, Od, collapse_ctr=ctr_d[0:1], collapse_sink_ctr=ctr_d[1:2],
+                    collapse_rows=rows_d, **kw)
+    torch.cuda.synchronize()
+    host = [t.cpu() for t in (Qg, Kg, Vg)]
+    if pinned:
+        host = [t.pin_memory() for t in host]
+    plan = HostPlan()
+    for chunks in (4, 5):   # pieces of one or two kv heads; first pieces split per head
+        ws = torch.empty(host_workspace_bytes(host_chunks=chunks, **{k: kw[k] for k in
+                         ("B", "H", "H_kv", "N", "d")}, qk_dtype=kw["qk_dtype"],
+                         o_dtype=kw["o_dtype"]), dtype=torch.uint8, device=dev)
+        side = torch.cuda.Stream()
+        for _ in range(2):
+            Oh = torch.full((B, H, N, d), float("nan"), dtype=o_dt)
+            if pinned:
+                Oh = Oh.pin_memory()
+            ctr = torch.zeros(2, dtype=torch.int64, device=dev)
+            rows = torch.full((B, H, N), -1, dtype=torch.int32, device=dev)
+            side.wait_stream(torch.cuda.current_stream())
+            fp8_attn_fwd_host(*host, Oh, plan=plan, workspace=ws, host_chunks=chunks,
+                              stream=side, collapse_ctr=ctr[0:1], collapse_sink_ctr=ctr[1:2],
+                              collapse_rows=rows, **kw)
+            side.synchronize()
+            assert torch.equal(Oh, Od.cpu())
+            assert torch.equal(ctr.cpu(), ctr_d.cpu())
+            assert torch.equal(rows.cpu(), rows_d.cpu())
+    plan.close()
+
+
 def test_empty_problems_are_a_no_op():
     """B, H or N of zero: the call succeeds, launches nothing and leaves the
     counters alone; attention() returns an empty O for device and host inputs."""
