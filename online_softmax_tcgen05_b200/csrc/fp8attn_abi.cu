@@ -135,7 +135,7 @@ bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int
 
 extern "C" {
 
-int fp8attn_version(void) { return 101; }
+int fp8attn_version(void) { return 102; }
 
 size_t fp8attn_params_sizeof(void) { return sizeof(fp8attn_params); }
 

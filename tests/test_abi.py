@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_params_layout(lib):
     assert lib.fp8attn_params_sizeof() == ctypes.sizeof(Params)
-    assert lib.fp8attn_version() == 101
+    assert lib.fp8attn_version() == 102
 
 
 def test_status_strings(lib):
