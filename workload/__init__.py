@@ -35,7 +35,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-__all__ = ["SinkWorkload", "make_sink_workload", "normals", "uniforms",
+__all__ = ["SinkWorkload", "make_sink_workload", "normals", "uniforms", "splitmix64",
            "ideal_logits", "CONFIG_SEED_BASE"]
 
 # Per-configuration seeds are CONFIG_SEED_BASE + configuration number.
@@ -68,8 +68,16 @@ def _load():
         u64 = ctypes.c_uint64
         lib.wl_normals.argtypes = [u64, u64, u64, u64, ctypes.c_void_p]
         lib.wl_uniforms.argtypes = [u64, u64, u64, u64, ctypes.c_void_p]
+        lib.wl_splitmix64.argtypes = [u64, u64, ctypes.c_void_p]
         _lib = lib
     return _lib
+
+
+def splitmix64(state: int, count: int) -> np.ndarray:
+    """The first `count` raw SplitMix64 outputs of the generator started at `state`."""
+    out = np.empty(count, dtype=np.uint64)
+    _load().wl_splitmix64(state, count, out.ctypes.data)
+    return out
 
 
 def uniforms(seed: int, stream: int, start: int, count: int) -> np.ndarray:

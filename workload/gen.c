@@ -39,3 +39,10 @@ void wl_normals(uint64_t seed, uint64_t stream, uint64_t start, uint64_t count, 
         out[i] = (float)((e & 1) ? r * sin(th) : r * cos(th));
     }
 }
+
+/* Raw SplitMix64 outputs from an explicit state: out[i] is the (i+1)-th output
+ * of the generator started at `state` (the sequence unif() draws from, before
+ * the top 53 bits are kept). */
+void wl_splitmix64(uint64_t state, uint64_t count, uint64_t* out) {
+    for (uint64_t i = 0; i < count; ++i) out[i] = mix64(state + (i + 1) * 0x9E3779B97F4A7C15ULL);
+}
