@@ -17,8 +17,8 @@ import math
 import numpy as np
 import pytest
 
-from helpers import (COLLAPSE_ABS, assert_o_close, compare_o, gpu_inputs, gpu_inputs_bf16, oracle,
-                     sample_rows, workload)
+from helpers import (COLLAPSE_ABS, assert_o_close, gpu_inputs, gpu_inputs_bf16, oracle, sample_rows,
+                     workload)
 
 pytestmark = pytest.mark.gpu
 

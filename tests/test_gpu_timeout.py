@@ -5,7 +5,6 @@ the kernel must then record where in the status word, free its TMEM and
 return, leaving the context usable for the next launch."""
 import math
 
-import numpy as np
 import pytest
 
 from helpers import assert_o_close, gpu_inputs, oracle, workload

@@ -14,7 +14,6 @@ Pins (P-E):
 * BF16 rounding against torch's float32 -> bfloat16 conversion.
 """
 import json
-import math
 import os
 
 import numpy as np
