@@ -119,7 +119,8 @@ def fp8_e4m3_scale_cast(P, out, S: float = 1.0, stream=None):
 
 def fp8_attn_fwd(Q, K, V, O, B, H, N, d, causal, scale, S, kv_order, n_sink, collapse_ctr=None,
                  stream=None):
-    """Direct call of the spec entry point (all tensors on the device)."""
+    """Direct call of the short entry point fp8_attn_fwd (H_kv = H, BF16 O, 128-key
+    blocks; all tensors on the device)."""
     _check(load_library().fp8_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, N, d,
                                        int(causal), float(scale), float(S), int(kv_order),
                                        int(n_sink), _ptr(collapse_ctr), _stream(stream)),
