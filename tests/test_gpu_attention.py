@@ -119,6 +119,36 @@ def test_parity_shapes(B, H, Hkv, N, d, block_n, causal):
                        what=(B, H, Hkv, N, d, block_n, causal, S, order))
 
 
+@pytest.mark.parametrize("case", range(16))
+def test_random_shapes(case):
+    """Seeded random problems: batch, GQA group, ragged N, d, block_n, causal or not,
+    order, S (powers of two and not), sink count, Delta and O dtype, all against
+    the oracle on every row."""
+    rng = np.random.default_rng(1000 + case)
+    Hkv = int(rng.integers(1, 4))
+    group = int(rng.choice([1, 2, 4, 5]))
+    B = int(rng.integers(1, 4))
+    while B * Hkv * group > 16:
+        B -= 1
+    if B == 0:
+        B, group = 1, 1
+    H = Hkv * group
+    N = int(rng.integers(1, 1501))
+    d = int(rng.choice([64, 128]))
+    block_n = int(rng.choice([64, 128]))
+    causal = int(rng.integers(0, 2))
+    order = int(rng.integers(0, 2))
+    S = float(rng.choice([0.5, 1.0, 16.0, 256.0, 300.0, 448.0]))
+    n_sink = int(rng.integers(0, min(N, 8) + 1))
+    delta = float(rng.uniform(0.0, 12.0))
+    f32 = bool(rng.integers(0, 2))
+    W = workload.make_sink_workload(B, H, Hkv, N, d, n_sink, delta, seed=5000 + case)
+    ins = gpu_inputs(W)
+    check_case(W, ins, causal, S, order, block_n, f32=f32,
+               what=dict(B=B, H=H, Hkv=Hkv, N=N, d=d, block_n=block_n, causal=causal,
+                         order=order, S=S, n_sink=n_sink, delta=delta, f32=f32))
+
+
 @pytest.mark.parametrize("N", [1, 2, 63, 127, 128, 129, 255])
 @pytest.mark.parametrize("causal", [0, 1])
 def test_edge_lengths(N, causal):
