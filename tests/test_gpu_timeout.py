@@ -39,3 +39,39 @@ def test_expired_wait_reports_status_and_context_survives():
     assert int(status.item()) == 0
     Oe, _, _ = oracle.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, 1 / math.sqrt(d), 256.0, 1, 128, 4)
     assert_o_close(O.cpu().numpy().reshape(-1, d), Oe, "after timeout")
+
+
+def test_host_entry_reports_expired_wait_and_recovers():
+    """The same failure through the host-buffer entry: the call returns, the
+    status word (a device word) records the expired wait once the caller's
+    stream has passed the call, and the next call on the same plan and
+    workspace is correct."""
+    import torch
+    from online_softmax_tcgen05_b200 import (O_F32, HostPlan, device_status_string,
+                                             fp8_attn_fwd_host, host_workspace_bytes)
+    B, H, Hkv, N, d = 1, 2, 1, 512, 128
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 8.0, seed=10)
+    ins = gpu_inputs(W)
+    (_, Q8), (_, K8), (_, V8) = ins
+    host = [torch.from_numpy(x).pin_memory() for x in (Q8, K8, V8)]
+    shape = dict(B=B, H=H, H_kv=Hkv, N=N, d=d)
+    plan = HostPlan()
+    ws = torch.empty(host_workspace_bytes(o_dtype=O_F32, host_chunks=1, **shape),
+                     dtype=torch.uint8, device="cuda")
+    O = torch.zeros((B, H, N, d), dtype=torch.float32).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kw = dict(S=256.0, kv_order=1, n_sink=4, o_dtype=O_F32, status_word=status, **shape)
+    fp8_attn_fwd_host(*host, O, plan=plan, workspace=ws, host_chunks=1, timeout_ns=50_000_000,
+                      debug_skip_kv_step=2, **kw)
+    torch.cuda.synchronize()
+    word = int(status.item())
+    assert (word & ~0xFF) == 0x100 and (word & 0xFF) != 0, hex(word)
+    assert device_status_string(word).startswith("timeout")
+    status.zero_()
+    fp8_attn_fwd_host(*host, O, plan=plan, workspace=ws, host_chunks=1, **kw)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    Oe, _, _ = oracle.attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, 0, 1 / math.sqrt(d), 256.0, 1, 128,
+                                   4)
+    assert_o_close(O.numpy().reshape(-1, d), Oe, "host entry after timeout")
+    plan.close()
