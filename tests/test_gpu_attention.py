@@ -142,11 +142,26 @@ def test_random_shapes(case):
     n_sink = int(rng.integers(0, min(N, 8) + 1))
     delta = float(rng.uniform(0.0, 12.0))
     f32 = bool(rng.integers(0, 2))
+    qk_bf16 = bool(rng.random() < 0.3)      # kernel-faithful mode: BF16 Q and K
+    cast_denominator = bool(rng.random() < 0.3)
+    what = dict(B=B, H=H, Hkv=Hkv, N=N, d=d, block_n=block_n, causal=causal, order=order, S=S,
+                n_sink=n_sink, delta=delta, f32=f32, qk_bf16=qk_bf16,
+                cast_denominator=cast_denominator)
     W = workload.make_sink_workload(B, H, Hkv, N, d, n_sink, delta, seed=5000 + case)
-    ins = gpu_inputs(W)
-    check_case(W, ins, causal, S, order, block_n, f32=f32,
-               what=dict(B=B, H=H, Hkv=Hkv, N=N, d=d, block_n=block_n, causal=causal,
-                         order=order, S=S, n_sink=n_sink, delta=delta, f32=f32))
+    ins = gpu_inputs_bf16(W) if qk_bf16 else gpu_inputs(W)
+    if not cast_denominator:
+        check_case(W, ins, causal, S, order, block_n, f32=f32, what=what)
+        return
+    (_, Q8), (_, K8), (_, V8) = ins
+    Og, _, _, crow = run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, n_sink, f32,
+                             denominator=1)
+    Oe, cr, _ = oracle.attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, W.scale, S, order,
+                                    block_n, n_sink, o_bf16=not f32, denom_mode=1)
+    assert np.isfinite(Og).all(), what
+    assert_o_close(Og, Oe, what)
+    denom = np.array([(r % N + 1 if causal else N) for r in range(B * H * N)], dtype=np.float64)
+    dfrac = np.abs(crow - cr.astype(np.int64)) / np.maximum(denom - n_sink, 1)
+    assert dfrac.max() <= COLLAPSE_ABS, (what, dfrac.max())
 
 
 @pytest.mark.parametrize("N", [1, 2, 63, 127, 128, 129, 255])
