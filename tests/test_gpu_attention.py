@@ -119,7 +119,7 @@ def test_parity_shapes(B, H, Hkv, N, d, block_n, causal):
                        what=(B, H, Hkv, N, d, block_n, causal, S, order))
 
 
-@pytest.mark.parametrize("case", range(16))
+@pytest.mark.parametrize("case", range(40))
 def test_random_shapes(case):
     """Seeded random problems: batch, GQA group, ragged N, d, block_n, causal or not,
     order, S (powers of two and not), sink count, Delta and O dtype, all against
