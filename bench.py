@@ -635,6 +635,69 @@ def report_batched_orders(dev):
                           "TFLOP/s": round(flops / ms / 1e9, 1)}), flush=True)
 
 
+def report_e2e_timeline(dev, steps=2, warmup=4):
+    """The prefill end to end through the host-buffer entry, profiled with CUPTI
+    (torch.profiler) for diagnosis: per step, the time from the step's first
+    device operation to its first kernel, the span from the first kernel's start
+    to the last kernel's end, the download tail after the last kernel, and the
+    bytes and busy time of the copies in each direction.  Times taken under a
+    profiler; never a bench value."""
+    import json as _json
+    import tempfile
+
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    import online_softmax_tcgen05_b200 as fa
+    cfg = CFG
+    W, (q, k, v) = make_inputs(rank_seed(0), dev)
+    B, H, N, d = W.B, W.H, W.N, W.d
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+
+    def step():
+        fa.attention(qh, kh, vh, causal=True, scale=1.0 / math.sqrt(d), S=cfg["S"],
+                     kv_order=cfg["kv_order"], n_sink=cfg["n_sink"], block_n=cfg["block_n"],
+                     count_collapse=True, out=oh)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(steps):
+            torch.cuda.synchronize()
+            step()
+        torch.cuda.synchronize()
+    with tempfile.NamedTemporaryFile(suffix=".json") as f:
+        prof.export_chrome_trace(f.name)
+        events = _json.load(open(f.name))["traceEvents"]
+    ev = sorted((e for e in events if e.get("ph") == "X" and e.get("cat") in
+                 ("kernel", "gpu_memcpy", "gpu_memset")), key=lambda e: e["ts"])
+    # each call starts by zeroing its collapse counters (a fill kernel): split there
+    starts = [i for i, e in enumerate(ev) if e["cat"] == "kernel" and "attn_fwd" not in e["name"]]
+    bounds = starts[:steps] + [len(ev)]
+    for sidx in range(len(bounds) - 1):
+        part = ev[bounds[sidx]:bounds[sidx + 1]]
+        kern = [e for e in part if e["cat"] == "kernel" and "attn_fwd" in e["name"]]
+        h2d = [e for e in part if e["cat"] == "gpu_memcpy" and "HtoD" in e["name"]]
+        d2h = [e for e in part if e["cat"] == "gpu_memcpy" and "DtoH" in e["name"]]
+        t0 = part[0]["ts"]
+        end = max(e["ts"] + e["dur"] for e in part)
+        k0 = min(e["ts"] for e in kern)
+        k1 = max(e["ts"] + e["dur"] for e in kern)
+        nbytes = lambda es: sum(int(e.get("args", {}).get("bytes", 0)) for e in es)
+        busy = lambda es: sum(e["dur"] for e in es) / 1e3
+        print(json.dumps({"report": "e2e-timeline", "step": sidx,
+                          "total_ms": round((end - t0) / 1e3, 3),
+                          "to_first_kernel_ms": round((k0 - t0) / 1e3, 3),
+                          "kernel_span_ms": round((k1 - k0) / 1e3, 3),
+                          "tail_after_last_kernel_ms": round((end - k1) / 1e3, 3),
+                          "kernels": len(kern),
+                          "h2d": {"copies": len(h2d), "MB": round(nbytes(h2d) / 1e6, 1),
+                                  "busy_ms": round(busy(h2d), 3)},
+                          "d2h": {"copies": len(d2h), "MB": round(nbytes(d2h) / 1e6, 1),
+                                  "busy_ms": round(busy(d2h), 3)}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -647,7 +710,8 @@ def main():
                          "the long-context problem split by kv heads (strong scaling)")
     ap.add_argument("--mode", choices=["full", "kernel"], default="full",
                     help="kernel: only the device-timed kernel loop (for profiling)")
-    ap.add_argument("--report", choices=["collapse", "configs", "batched-orders"], default=None,
+    ap.add_argument("--report", choices=["collapse", "configs", "batched-orders", "e2e-timeline"],
+                    default=None,
                     help="one GPU: JSON lines for the Delta/S collapse sweep against the closed "
                          "form, or the timing protocols of the larger configurations")
     args = ap.parse_args()
@@ -656,7 +720,8 @@ def main():
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         {"collapse": report_collapse, "configs": report_configs,
-         "batched-orders": report_batched_orders}[args.report](dev)
+         "batched-orders": report_batched_orders,
+         "e2e-timeline": report_e2e_timeline}[args.report](dev)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
