@@ -103,6 +103,12 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     scale = scale if scale is not None else 1.0 / math.sqrt(d)
     kw = dict(causal=causal, scale=scale, S=S, kv_order=kv_order, n_sink=n_sink,
               block_n=block_n, denominator=denominator, o_code=o_code)
+    if out is not None:
+        if (tuple(out.shape) != (B, H, N, d) or out.dtype != out_dtype
+                or not out.is_contiguous()
+                or (out.device != q.device if q.is_cuda else out.device.type != "cpu")):
+            raise ValueError("out must be a contiguous %s tensor of shape %s on %s"
+                             % (out_dtype, (B, H, N, d), q.device))
     stats = AttentionStats()
     if B * H * N == 0:   # nothing to compute: an empty O (per-row counts empty too)
         import torch

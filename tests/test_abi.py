@@ -140,3 +140,18 @@ def test_host_entry_rejects_before_any_cuda_call(lib, kw, plan, ws, nbytes, chun
     st = lib.fp8_attn_fwd_host(ctypes.byref(p), plan, ws, nbytes, chunks, None)
     assert st in (EINVAL, EUNSUPPORTED)
     assert _binding.last_error() != ""
+
+
+@pytest.mark.parametrize("bad", ["shape", "dtype", "layout", "device"])
+def test_attention_rejects_unusable_out(bad):
+    # checked before any copy or launch, so host tensors suffice (no GPU)
+    import torch
+    from online_softmax_tcgen05_b200 import attention
+    B, H, N, d = 1, 2, 128, 64
+    q = torch.zeros((B, H, N, d), dtype=torch.uint8)
+    out = {"shape": torch.empty((B, H, N + 1, d), dtype=torch.bfloat16),
+           "dtype": torch.empty((B, H, N, d), dtype=torch.float32),
+           "layout": torch.empty((B, H, d, N), dtype=torch.bfloat16).transpose(2, 3),
+           "device": torch.empty((B, H, N, d), dtype=torch.bfloat16, device="meta")}[bad]
+    with pytest.raises(ValueError):
+        attention(q, q, q, out=out)
