@@ -240,8 +240,10 @@ def test_host_tensors_many_chunks(chunks):
     assert torch.equal(st_h.collapse_rows.cpu(), st_d.collapse_rows.cpu())
 
 
-@pytest.mark.parametrize("qk_bf16,o_f32,pinned", [(False, False, True), (True, True, False)])
-def test_host_entry_direct(qk_bf16, o_f32, pinned):
+@pytest.mark.parametrize("qk_bf16,o_f32,pinned,causal", [(False, False, True, 1),
+                                                         (True, True, False, 1),
+                                                         (False, True, True, 0)])
+def test_host_entry_direct(qk_bf16, o_f32, pinned, causal):
     """fp8_attn_fwd_host called directly on a side stream, twice with one plan and
     workspace (the second call reuses every staging set): O, the counters and the
     per-row counts equal the device entry's bit for bit, with pinned or pageable
@@ -258,7 +260,7 @@ def test_host_entry_direct(qk_bf16, o_f32, pinned):
         ins = gpu_inputs(W)
     (Qg, _), (Kg, _), (Vg, _) = ins
     o_dt = torch.float32 if o_f32 else torch.bfloat16
-    kw = dict(B=B, H=H, H_kv=Hkv, N=N, d=d, causal=1, S=256.0, kv_order=1, n_sink=4,
+    kw = dict(B=B, H=H, H_kv=Hkv, N=N, d=d, causal=causal, S=256.0, kv_order=1, n_sink=4,
               o_dtype=O_F32 if o_f32 else O_BF16, qk_dtype=QK_BF16 if qk_bf16 else QK_E4M3)
     dev = Qg.device
     Od = torch.empty((B, H, N, d), dtype=o_dt, device=dev)
