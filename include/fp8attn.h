@@ -186,6 +186,44 @@ size_t fp8attn_host_workspace_bytes(const fp8attn_params* p, int host_chunks);
 int fp8_attn_fwd_host(const fp8attn_params* p, fp8attn_host_plan* plan, void* workspace,
                       size_t workspace_bytes, int host_chunks, fp8attn_stream_t stream);
 
+/* ------------------------------------------ host-buffer entry, no allocation ---
+ * fp8_attn_fwd_host_noalloc - the same operation as fp8_attn_fwd_host for a
+ * caller that cannot allocate device memory: code running where another
+ * allocator owns the whole device (a plugin inside a host application, a
+ * framework that reserves all of HBM up front), a serving loop whose rules
+ * forbid allocation after start-up, or a plain C caller with no CUDA allocator
+ * of its own.  It takes no workspace and no plan and calls no allocating
+ * routine (no cudaMalloc, cudaFree, stream or event creation).  The P-cast
+ * paper has no counterpart: this is a deployment convenience of the library.
+ *
+ * Staging goes through one array of FP8ATTN_HOST_NOALLOC_BYTES bytes of device
+ * memory that the library holds as a static device variable: every GPU that
+ * loads the library's module holds it until the process exits.  The problem is
+ * cut into pieces of whole (batch, kv-head) units, as many kv heads of one
+ * batch element as fit the array; each piece's copies in, its kernel and its
+ * copy back run in order on `stream` (no overlap of copies and kernels; the
+ * pipelined fp8_attn_fwd_host is the fast path).
+ *
+ *   p       as for fp8_attn_fwd_host: Q, K, V, O are HOST pointers; the
+ *           collapse counters, per-row counts and status word stay DEVICE
+ *           pointers; q_begin = q_end = 0.
+ *   stream  the call's work runs in order on it, after prior work; synchronise
+ *           it before reading O or the counters.
+ * Returns an fp8attn_status.  FP8ATTN_EINVAL, with fp8attn_last_error() giving
+ * the sizes, when one kv head's Q, K, V and O (H / H_kv query heads) need more
+ * than FP8ATTN_HOST_NOALLOC_BYTES of staging, rounded up to 256 bytes per buffer.
+ *
+ * The first call on a device, with that device current, looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls share the one array, which keeps the last call's contents
+ * (a call reads only staging bytes it wrote first, so nothing needs clearing).
+ * Calls that overlap on the GPU (different streams, or several host threads
+ * without ordering between their streams) race on it: order them, for instance
+ * by issuing them all on one stream. */
+#define FP8ATTN_HOST_NOALLOC_BYTES ((size_t)64 << 20)
+
+int fp8_attn_fwd_host_noalloc(const fp8attn_params* p, fp8attn_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fp8attn_status_string(int status);
 

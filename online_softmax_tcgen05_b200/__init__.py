@@ -20,11 +20,11 @@ from dataclasses import dataclass
 from ._binding import (DENOM_CAST_P, DENOM_FP32_P, ECUDA, EINVAL, ETIMEOUT, EUNSUPPORTED,
                        KV_FORWARD, KV_REVERSE, O_BF16, O_F32, OK, QK_BF16, QK_E4M3, Fp8AttnError,
                        HostPlan, device_status_string, fp8_attn_fwd, fp8_attn_fwd_ex,
-                       fp8_attn_fwd_host, fp8_e4m3_scale_cast, host_workspace_bytes, last_error,
-                       load_library, status_string)
+                       fp8_attn_fwd_host, fp8_attn_fwd_host_noalloc, fp8_e4m3_scale_cast,
+                       host_workspace_bytes, last_error, load_library, status_string)
 
 __all__ = ["attention", "AttentionStats", "fp8_attn_fwd", "fp8_attn_fwd_ex",
-           "fp8_attn_fwd_host", "HostPlan", "host_workspace_bytes",
+           "fp8_attn_fwd_host", "fp8_attn_fwd_host_noalloc", "HostPlan", "host_workspace_bytes",
            "fp8_e4m3_scale_cast", "load_library", "status_string", "last_error",
            "device_status_string", "Fp8AttnError", "KV_FORWARD", "KV_REVERSE", "O_BF16",
            "O_F32", "OK", "EINVAL", "EUNSUPPORTED", "ECUDA", "ETIMEOUT", "e4m3_cast",

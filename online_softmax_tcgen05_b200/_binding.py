@@ -58,6 +58,7 @@ SIGNATURES = {
     "fp8attn_host_workspace_bytes": ([ctypes.POINTER(Params), ctypes.c_int], ctypes.c_size_t),
     "fp8_attn_fwd_host": ([ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_void_p,
                            ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
+    "fp8_attn_fwd_host_noalloc": ([ctypes.POINTER(Params), ctypes.c_void_p], ctypes.c_int),
 }
 
 _lib = None
@@ -197,3 +198,18 @@ def fp8_attn_fwd_host(Q, K, V, O, *, plan, workspace, host_chunks=16, stream=Non
                                             ctypes.c_void_p(workspace.data_ptr()), nbytes,
                                             int(host_chunks), _stream(stream)),
            "fp8_attn_fwd_host")
+
+
+# FP8ATTN_HOST_NOALLOC_BYTES of include/fp8attn.h: the staging array of
+# fp8_attn_fwd_host_noalloc
+HOST_NOALLOC_BYTES = 64 << 20
+
+
+def fp8_attn_fwd_host_noalloc(Q, K, V, O, *, stream=None, **kw):
+    """Host-buffer entry point that allocates nothing: Q, K, V, O are CPU
+    tensors, counters and per-row counts CUDA tensors; staging goes through the
+    library's own fixed device array (HOST_NOALLOC_BYTES).  Runs in order on
+    ``stream`` (default: current); synchronise it before reading O."""
+    p = _params(Q, K, V, O, **kw)
+    _check(load_library().fp8_attn_fwd_host_noalloc(ctypes.byref(p), _stream(stream)),
+           "fp8_attn_fwd_host_noalloc")
