@@ -11,7 +11,11 @@
  * is a run-time choice; section 2 "Optimisation 1" shows that the reverse order
  * keeps the attention sink from inflating m before the other blocks are cast.
  * "P-collapse" (section 1) is a non-sink P that is nonzero in FP32 but 0 after
- * the cast; the kernel can count it.
+ * the cast; the kernel can count it.  What the kernel counts: every visible
+ * non-sink key (j >= n_sink, and j <= i when causal) whose E4M3 byte of S*p is
+ * zero.  That equals "p_j > 0 in FP32 and zero after the cast" except where the
+ * FP32 p_j itself is 0 (s_j - m' below about -87 nats, where ex2 flushes to
+ * zero): such a key is counted here although its FP32 value is not nonzero.
  *
  * Per query row i (query head h, kv head h / (H / H_kv)):
  *   for each KV block of block_n keys, in the chosen order:
@@ -23,6 +27,10 @@
  *     acc  = alpha * acc + sum_j pt_j v_j   (E4M3 x E4M3, FP32 accumulate)
  *     m    = m'
  *   O_i = acc / (S * l)
+ * For S a power of two the kernel takes S * p_j directly from its exponential,
+ * 2^(log2 e * (s_j - m') + log2 S), and sums those, so S divides out with l:
+ * the same real numbers, exact scaling.  For any other S it forms the FP32
+ * product fl(S * p_j) that is cast, sums the p_j, and divides by fl(S * l).
  * Causal: key j is visible to query i iff j <= i (square prefill, no offset).
  *
  * Conventions for every entry point:
@@ -84,7 +92,8 @@ enum { FP8ATTN_DENOM_FP32_P = 0, FP8ATTN_DENOM_CAST_P = 1 };
  *   n_sink    keys j < n_sink are sinks and are never counted (0 <= n_sink <= N).
  *   collapse_ctr  NULL: no counting (the faster kernel variant).  Otherwise a
  *             device uint64 that the kernel ADDS the number of collapsed
- *             entries to (the caller zeroes it).
+ *             entries to (the caller zeroes it): visible non-sink keys whose
+ *             E4M3 byte of S*p is zero (see "What the kernel counts" above).
  * Returns an fp8attn_status. */
 int fp8_attn_fwd(const void* Q, const void* K, const void* V, void* O,
                  int B, int H, int N, int d, int causal, float scale, float S,
@@ -116,7 +125,11 @@ typedef struct {
   unsigned int* status_word;             /* nullable device word; a kernel whose bounded
                                             wait expires writes a nonzero code here and
                                             leaves O incomplete */
-  unsigned long long timeout_ns;         /* bound of each wait; 0 = 2 s */
+  unsigned long long timeout_ns;         /* bound of each wait: 0 = 2 s, otherwise at
+                                            least 1 ms (1000000); smaller values are
+                                            rejected.  After an expired wait the CTA
+                                            still waits up to 1 s for its own copies
+                                            and MMAs in flight before it exits. */
   int debug_skip_kv_step;                /* testing only, normally 0.  k > 0: the producer
                                             never issues the K tile of the k-th KV step
                                             (1-based), so the MMA warp's bounded wait runs
@@ -134,10 +147,13 @@ typedef struct {
 
 int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream);
 
-/* fp8_e4m3_scale_cast - out[i] = E4M3_RNE_satfinite(fl32(S * P[i])) for i < n,
- * with the device conversion routine the attention kernel uses for S*P
- * (P-cast paper, section 2 "Optimality of S=256": the scaling happens in FP32,
- * then the round-to-nearest cast).  P: device float[n]; out: device uint8[n];
+/* fp8_e4m3_scale_cast - out[i] = E4M3_RNE_satfinite(fl32(S * P[i])) for i < n:
+ * one FP32 multiply, then the conversion instruction (cvt.rn.satfinite.e4m3x2)
+ * that the attention kernel applies to S*p (P-cast paper, section 2
+ * "Optimality of S=256": the scaling happens in FP32, then the round-to-nearest
+ * cast).  For S not a power of two the attention kernel forms S*p by the same
+ * FP32 multiply; for S = 2^k it takes S*p from its exponential and never forms
+ * the product, which for finite p without over- or underflow is the same value.  P: device float[n]; out: device uint8[n];
  * both 16-byte aligned.  S finite (any sign).  NaN -> 0x7F, |x| > 448 -> +-448. */
 int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
                         fp8attn_stream_t stream);
@@ -168,7 +184,9 @@ int fp8_e4m3_scale_cast(const float* P, unsigned char* out, size_t n, float S,
  *                ordered after the last copy back: synchronise it before reading
  *                O or the counters.
  * Returns an fp8attn_status.  A failure after work was enqueued (FP8ATTN_ECUDA)
- * leaves O incomplete and the plan's streams possibly busy. */
+ * leaves O incomplete; `stream` is still ordered after all work the call
+ * enqueued (unless the CUDA context itself has failed), so the workspace and
+ * the host buffers may be released once `stream` has passed the call. */
 typedef struct fp8attn_host_plan fp8attn_host_plan;   /* opaque */
 
 /* Streams and events of the host pipeline, on the current device.  A plan

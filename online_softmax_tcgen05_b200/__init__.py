@@ -87,7 +87,11 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
     piece's upload, kernels and download against its neighbours'.  Pinned host
     memory makes the copies asynchronous.  ``stream`` (default: the current
     stream) is ordered before and after the whole call, which returns once O is
-    in host memory."""
+    in host memory.
+
+    CUDA tensors: q, k, v (and ``out``) must share one device; the kernel runs
+    there on ``stream`` (default: that device's current stream), ordered after
+    the device's current stream, which in turn waits for the kernel."""
     import torch
     q, k, v = _as_bytes(q, True), _as_bytes(k, True), _as_bytes(v)
     if (q.dtype == torch.bfloat16) != (k.dtype == torch.bfloat16):
@@ -109,6 +113,15 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
                 or (out.device != q.device if q.is_cuda else out.device.type != "cpu")):
             raise ValueError("out must be a contiguous %s tensor of shape %s on %s"
                              % (out_dtype, (B, H, N, d), q.device))
+    if q.is_cuda or k.is_cuda or v.is_cuda:
+        devs = {t.device for t in (q, k, v)}
+        if out is not None:
+            devs.add(out.device)
+        if len(devs) != 1 or q.device.type != "cuda":
+            raise ValueError("q, k, v (and out) must all be on one CUDA device, got %s"
+                             % sorted(str(x) for x in devs))
+        if stream is not None and stream.device != q.device:
+            raise ValueError("stream is on %s, the tensors on %s" % (stream.device, q.device))
     stats = AttentionStats()
     if B * H * N == 0:   # nothing to compute: an empty O (per-row counts empty too)
         import torch
@@ -118,17 +131,30 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, S: f
             stats.collapse_rows = torch.zeros((B, H, N), dtype=torch.int32, device=dev)
         return o, stats
     if q.is_cuda:
-        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        # The library launches on the current device and on `s`; the tensors made
+        # here come from the caching allocator on the current stream `cur`.
         dev = q.device
-        o = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype, device=dev)
-        ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
-        rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
-                if (count_collapse and per_row) else None)
-        _launch(q, k, v, o, ctr, rows, stream=stream, **kw)
-        if ctr is not None:
-            c = ctr.cpu()
-            stats.collapse, stats.collapse_sink_block = int(c[0]), int(c[1])
-            stats.collapse_rows = rows
+        with torch.cuda.device(dev):
+            cur = torch.cuda.current_stream(dev)
+            s = cur if stream is None else stream
+            q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+            o = out if out is not None else torch.empty((B, H, N, d), dtype=out_dtype,
+                                                        device=dev)
+            ctr = torch.zeros(2, dtype=torch.int64, device=dev) if count_collapse else None
+            rows = (torch.zeros((B, H, N), dtype=torch.int32, device=dev)
+                    if (count_collapse and per_row) else None)
+            if s is not cur:
+                s.wait_stream(cur)   # the copies and zeroed counters above, on cur
+            _launch(q, k, v, o, ctr, rows, stream=s, **kw)
+            if s is not cur:
+                for t in (q, k, v, o, ctr, rows):
+                    if t is not None:
+                        t.record_stream(s)
+                cur.wait_stream(s)   # the counters are read on cur below
+            if ctr is not None:
+                c = ctr.cpu()
+                stats.collapse, stats.collapse_sink_block = int(c[0]), int(c[1])
+                stats.collapse_rows = rows
         return o, stats
 
     # ---- host tensors: the library's host-buffer pipeline (fp8_attn_fwd_host) ----

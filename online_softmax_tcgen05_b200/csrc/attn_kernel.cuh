@@ -14,6 +14,11 @@ namespace fp8attn {
 
 constexpr int BM = 128;         // query rows per CTA (= MMA M, = TMEM lanes)
 constexpr float LOG2E = 1.4426950408889634f;
+// Smallest nonzero bound of a wait the caller may set (timeout_ns), and the
+// fixed bound of the drain waits that let in-flight copies and MMAs land
+// before an aborting CTA frees TMEM and exits.
+constexpr unsigned long long MIN_TIMEOUT_NS = 1000000ull;
+constexpr unsigned long long DRAIN_TIMEOUT_NS = 1000000000ull;
 
 // device status codes (status_word): 0x100 | where the wait gave up
 enum : uint32_t {
@@ -33,9 +38,15 @@ struct KParams {
   int causal, kv_order, n_sink;
   int tile0;          // first query tile of the launch (q_begin / 128)
   int num_q_tiles;    // query tiles in the launch
-  int sched_group;    // (batch, head) planes per causal scheduling group; divides B * H
+  int sched_group;    // plane units per causal scheduling group; divides their number
+  int pair_heads;     // two-tile kernel: 1 = a CTA's tiles are one tile of two query
+                      // heads of one kv head, 0 = two consecutive tiles of one head
   float scale_log2;   // scale * log2(e)
-  float log2S;   // log2(S): S*p is taken as 2^(s*c - m + log2 S)
+  // S*p: for S = 2^k, log2S = k and s_mul = 1, S*p is taken as 2^(s*c - m + k)
+  // (exact scaling); otherwise log2S = 0 and S*p = fl(p * S) after the
+  // exponential, the FP32 product the method casts.
+  float log2S;
+  float s_mul;
   void* O;
   unsigned long long* ctr;
   unsigned long long* ctr_sink;
@@ -52,6 +63,13 @@ struct KParams {
 cudaError_t launch_attn(int d, int bn, bool o_bf16, bool count, bool qk_bf16,
                         const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                         const KParams& kp, cudaStream_t stream);
+
+// The same operation with two query tiles per CTA and one CTA per SM
+// (fp8_attn_fwd_pair.cu).  Grid: (row units, plane units): kp.pair_heads ?
+// (num_q_tiles, B * H / 2) : (ceil(num_q_tiles / 2), B * H).
+cudaError_t launch_attn_pair(int d, int bn, bool o_bf16, bool count, bool qk_bf16,
+                             const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                             const KParams& kp, cudaStream_t stream);
 
 // out[i] = E4M3_RNE_satfinite(fl32(S * P[i])), i < n (P, out 16-byte aligned).
 cudaError_t launch_e4m3_scale_cast(const float* P, uint8_t* out, size_t n, float S,

@@ -22,10 +22,13 @@
 //              N=block_n, K=32 per instruction), then O += P~ V into TMEM
 //              (V as an MN-major operand).  Owns the TMEM allocation.
 //   warps 0-3  softmax, one thread per query row: tcgen05.ld of its score row,
-//              row max, S*p as one exp2 with log2 S added to the argument, FP32
-//              row sum of S*p, E4M3 cast into a swizzled shared-memory P~ tile,
-//              collapse count, the O rescale in TMEM when a row max changed, and
-//              the epilogue O / l (l: the row sum of S*p, so S divides out).
+//              row max, exponentials, FP32 row sum, E4M3 cast of S*p into a
+//              swizzled shared-memory P~ tile, collapse count, the O rescale in
+//              TMEM when a row max changed, and the epilogue O / (S l).  For
+//              S = 2^k, S*p is one exp2 with k added to the argument and the row
+//              sum is of S*p (so S divides out with l); for any other S the
+//              kernel forms fl(S * p) with an FP32 multiply, as the method states,
+//              sums p, and divides by fl(S * l).
 // Every mbarrier wait is bounded in time: on expiry the CTA sets a shared
 // abort flag, every role leaves its loop, in-flight copies and MMAs are
 // drained, TMEM is freed and the status word (if given) records where.
@@ -213,7 +216,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // drain: the last load issued into each stage must land before the CTA
         // exits (immediate when the consumers took them all; needed after an abort)
         const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8),
-                            p.timeout_ns};
+                            DRAIN_TIMEOUT_NS};
         for (int t = k_issued - 1; t >= 0 && t >= k_issued - NSTAGE; --t)
           mbar_wait(bar_k_full(t % NSTAGE), (t / NSTAGE) & 1, drain, 0);
         for (int t = v_issued - 1; t >= 0 && t >= v_issued - NSTAGE; --t)
@@ -286,7 +289,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     if (!ok) {
       // drain every MMA this warp issued before TMEM is released
-      const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8), p.timeout_ns};
+      const WaitCtl drain{reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8),
+                          DRAIN_TIMEOUT_NS};
       if (lane == 0) mma_commit(bar_drain);
       __syncwarp();
       mbar_wait(bar_drain, 0, drain, 0);
@@ -323,11 +327,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float* s = reinterpret_cast<float*>(sr);
       const bool need_mask = (p.causal && j0 + BN - 1 > q0) || (j0 + BN > p.N);
       const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;   // last visible key
-      // Most blocks hold no masked key and no sink key and use the FP32 row sum:
-      // they take a copy of the block's arithmetic with no branch in it, so that
-      // the integer work of the cast and the count can interleave with the
-      // exponentials of the same block.
-      const bool plain = !need_mask && j0 >= p.n_sink && !p.denom_cast;
+      // Most blocks hold no masked key and no sink key and use the FP32 row sum
+      // and a power-of-two S: they take a copy of the block's arithmetic with no
+      // branch in it, so that the integer work of the cast and the count can
+      // interleave with the exponentials of the same block.
+      const bool plain = !need_mask && j0 >= p.n_sink && !p.denom_cast && p.s_mul == 1.f;
       float m_new, alpha;
       uint32_t pw[BN / 4];
       auto block_math = [&](auto plain_tag) {
@@ -358,8 +362,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m_new = fmaxf(m_run, mx * c);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-        // S*p = 2^(s*c - m + log2 S): packed FFMA2 for the argument, MUFU ex2,
-        // split row sums (of S*p: the epilogue scales O by 1 / that sum, S included)
+        // 2^(s*c - m + log2S): packed FFMA2 for the argument, MUFU ex2, split row
+        // sums.  For S = 2^k (log2S = k) that is S*p and its row sum carries S;
+        // otherwise (log2S = 0) it is p, multiplied by S below.
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
         float2 acc8[8];
 #pragma unroll
@@ -387,10 +392,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         } else {
           if (!p.denom_cast) l = alpha * l + rowsum;
         }
-        // the E4M3 cast of S*p, four keys per word
+        // the E4M3 cast of S*p, four keys per word.  Blocks off the plain path
+        // form fl(s_mul * x): the method's FP32 product S*p when S is not a power
+        // of two, an exact multiply by 1 when S*p came out of the exponential.
+        const float2 sm2 = make_float2(p.s_mul, p.s_mul);
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q)
-          pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+        for (int q = 0; q < BN / 4; ++q) {
+          if constexpr (PLAIN) {
+            pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+          } else {
+            const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), sm2);
+            const float2 b = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), sm2);
+            pw[q] = pack_e4m3x4(a.x, a.y, b.x, b.y);
+          }
+        }
         if constexpr (!PLAIN) {
           if (p.denom_cast) {
             // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
@@ -507,9 +522,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     if (ok) {
       tc_fence_after();
-      // O = acc * 1/l, l being the row sum of S*p (so S divides out here); one
-      // correctly rounded reciprocal per row, then a multiply per element
-      const float inv_l = __frcp_rn(l);
+      // O = acc / (S l): one correctly rounded reciprocal per row, then a
+      // multiply per element.  For S = 2^k, l already is the row sum of S*p
+      // (s_mul = 1); otherwise the denominator is fl(S * l).  The cast-value row
+      // sum carries S in its values.
+      const float inv_l = __frcp_rn(p.denom_cast ? l : l * p.s_mul);
       const bool live = row < p.N;
       const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
 #pragma unroll

@@ -15,6 +15,12 @@
 #include "attn_kernel.cuh"
 #include "fp8attn.h"
 
+// 1: the two-tile kernel (fp8_attn_fwd_pair.cu); 0: one tile per CTA
+// (fp8_attn_fwd.cu).  Same arithmetic, different schedule.
+#ifndef FP8ATTN_PAIR_KERNEL
+#define FP8ATTN_PAIR_KERNEL 0
+#endif
+
 namespace fp8attn {
 
 namespace {
@@ -53,6 +59,8 @@ int validate(const fp8attn_params* p, bool host_buffers) {
     return fail(FP8ATTN_EINVAL, "qk_dtype must be FP8ATTN_QK_E4M3 or FP8ATTN_QK_BF16");
   if (p->o_dtype != FP8ATTN_O_BF16 && p->o_dtype != FP8ATTN_O_F32)
     return fail(FP8ATTN_EINVAL, "o_dtype must be FP8ATTN_O_BF16 or FP8ATTN_O_F32");
+  if (p->timeout_ns != 0 && p->timeout_ns < MIN_TIMEOUT_NS)
+    return fail(FP8ATTN_EINVAL, "timeout_ns must be 0 (the 2 s default) or at least 1 ms");
   if (p->debug_skip_kv_step < 0) return fail(FP8ATTN_EINVAL, "debug_skip_kv_step must be >= 0");
   if (p->debug_skip_kv_step > 0 && !p->status_word)
     return fail(FP8ATTN_EINVAL, "debug_skip_kv_step needs a status_word to report the timeout");
@@ -135,7 +143,7 @@ bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int
 
 extern "C" {
 
-int fp8attn_version(void) { return 102; }
+int fp8attn_version(void) { return 103; }
 
 size_t fp8attn_params_sizeof(void) { return sizeof(fp8attn_params); }
 
@@ -201,6 +209,12 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
     while (nkv % kvg) --kvg;
     kp.sched_group = kvg * kp.group;
   }
+  // two-tile kernel: an even GQA group pairs two query heads of one kv head,
+  // otherwise two consecutive tiles of one head; its scheduling groups count
+  // plane units (head pairs or planes)
+  kp.pair_heads = (kp.group % 2 == 0) ? 1 : 0;
+  const bool use_pair = FP8ATTN_PAIR_KERNEL != 0;
+  if (use_pair && kp.pair_heads) kp.sched_group /= 2;
   kp.causal = p->causal;
   kp.kv_order = p->kv_order;
   kp.n_sink = p->n_sink;
@@ -211,7 +225,13 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
     kp.num_q_tiles = (r1 + fp8attn::BM - 1) / fp8attn::BM - kp.tile0;
   }
   kp.scale_log2 = p->scale * fp8attn::LOG2E;
-  kp.log2S = (float)std::log2((double)p->S);
+  {
+    // S = 2^k enters the exponent (exact scaling); any other S multiplies p
+    int e2 = 0;
+    const bool pow2 = std::frexp((double)p->S, &e2) == 0.5;
+    kp.log2S = pow2 ? (float)(e2 - 1) : 0.f;
+    kp.s_mul = pow2 ? 1.f : p->S;
+  }
   kp.O = p->O;
   kp.ctr = p->collapse_ctr;
   kp.ctr_sink = p->collapse_sink_ctr;
@@ -225,7 +245,9 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   const bool count = p->collapse_ctr != nullptr;
   const bool qk_bf16 = p->qk_dtype == FP8ATTN_QK_BF16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = fp8attn::launch_attn(p->d, bn, bf16, count, qk_bf16, mq, mk, mv, kp, s);
+  const cudaError_t e =
+      use_pair ? fp8attn::launch_attn_pair(p->d, bn, bf16, count, qk_bf16, mq, mk, mv, kp, s)
+               : fp8attn::launch_attn(p->d, bn, bf16, count, qk_bf16, mq, mk, mv, kp, s);
   if (e != cudaSuccess) return fail(FP8ATTN_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return FP8ATTN_OK;
 }

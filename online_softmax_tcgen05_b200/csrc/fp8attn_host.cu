@@ -97,6 +97,17 @@ int cuda_fail(cudaError_t e, const char* what) {
   return fail(FP8ATTN_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
 
+// A failure after work was enqueued on the plan's streams: before returning
+// `status`, order the caller's stream after everything those streams hold, so
+// that a caller who frees the workspace or the host buffers once its stream
+// has passed the call frees nothing a copy still uses.  Best effort: in a
+// context that has itself failed these calls fail too.
+int fail_joined(fp8attn_host_plan* pl, cudaStream_t caller, int status) {
+  for (cudaStream_t s : {pl->s_in, pl->s_out, pl->s_comp[0], pl->s_comp[1]})
+    if (cudaEventRecord(pl->ev_end, s) == cudaSuccess) cudaStreamWaitEvent(caller, pl->ev_end, 0);
+  return status;
+}
+
 }  // namespace
 
 extern "C" {
@@ -187,7 +198,7 @@ int fp8_attn_fwd_host(const fp8attn_params* p, fp8attn_host_plan* pl, void* work
   e = cudaEventRecord(pl->ev_start, caller);
   for (cudaStream_t s : {pl->s_in, pl->s_out, pl->s_comp[0], pl->s_comp[1]})
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, pl->ev_start, 0);
-  if (e != cudaSuccess) return cuda_fail(e, "stream ordering");
+  if (e != cudaSuccess) return fail_joined(pl, caller, cuda_fail(e, "stream ordering"));
 
   int step = 0;
   const int np = (int)pieces.size();
@@ -217,13 +228,13 @@ int fp8_attn_fwd_host(const fp8attn_params* p, fp8attn_host_plan* pl, void* work
                           (a1 - a0) * z.plane_qk, cudaMemcpyHostToDevice, pl->s_in);
       if (e == cudaSuccess) e = cudaEventRecord(pl->ev_in[j], pl->s_in);
     }
-    if (e != cudaSuccess) return cuda_fail(e, "upload");
+    if (e != cudaSuccess) return fail_joined(pl, caller, cuda_fail(e, "upload"));
 
     for (int j = 0; j < nsub; ++j) {
       const int a0 = split ? j : 0, a1 = split ? j + 1 : nq;
       cudaStream_t comp = pl->s_comp[step++ % 2];
       e = cudaStreamWaitEvent(comp, pl->ev_in[j], 0);
-      if (e != cudaSuccess) return cuda_fail(e, "stream ordering");
+      if (e != cudaSuccess) return fail_joined(pl, caller, cuda_fail(e, "stream ordering"));
       const size_t q_plane0 = (size_t)pc.b * p->H + hq + a0;
       fp8attn_params sub = *p;
       sub.Q = qd + a0 * z.plane_qk;
@@ -235,22 +246,22 @@ int fp8_attn_fwd_host(const fp8attn_params* p, fp8attn_host_plan* pl, void* work
       sub.H_kv = nk;
       sub.collapse_rows = p->collapse_rows ? p->collapse_rows + q_plane0 * p->N : nullptr;
       const int st = fp8_attn_fwd_ex(&sub, comp);
-      if (st != FP8ATTN_OK) return st;   // last error set by the launch
+      if (st != FP8ATTN_OK) return fail_joined(pl, caller, st);   // last error set by the launch
       e = cudaEventRecord(pl->ev_done, comp);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(pl->s_out, pl->ev_done, 0);
       if (e == cudaSuccess)
         e = cudaMemcpyAsync(Oh + q_plane0 * z.plane_o, od + a0 * z.plane_o,
                             (a1 - a0) * z.plane_o, cudaMemcpyDeviceToHost, pl->s_out);
-      if (e != cudaSuccess) return cuda_fail(e, "download");
+      if (e != cudaSuccess) return fail_joined(pl, caller, cuda_fail(e, "download"));
     }
     e = cudaEventRecord(pl->ev_free[set], pl->s_out);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if (e != cudaSuccess) return fail_joined(pl, caller, cuda_fail(e, "cudaEventRecord"));
     pl->free_recorded[set] = true;
   }
   // the caller's stream continues after the last download (and so after every kernel)
   e = cudaEventRecord(pl->ev_end, pl->s_out);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(caller, pl->ev_end, 0);
-  if (e != cudaSuccess) return cuda_fail(e, "stream ordering");
+  if (e != cudaSuccess) return fail_joined(pl, caller, cuda_fail(e, "stream ordering"));
   return FP8ATTN_OK;
 }
 

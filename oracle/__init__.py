@@ -67,10 +67,13 @@ def lib():
                                         i32]
         L.oracle_attn_exact.restype = i32
         L.oracle_attn_emulate.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f32, f32,
-                                          i32, i32, i32, i32, P, i64, P, P, P, i32, i32, i32]
+                                          i32, i32, i32, i32, P, i64, P, P, P, i32, i32, i32, P]
         L.oracle_attn_emulate.restype = i32
         L.oracle_collapse_logits.argtypes = [P, i64, i32, i32, i32, f32, i32, P, P, i32]
         L.oracle_collapse_logits.restype = i32
+        L.oracle_attn_logits.argtypes = [P, P, i64, i32, i32, i32, i32, i32, f32, i32, P, P, P,
+                                         i32]
+        L.oracle_attn_logits.restype = i32
         _lib = L
     return _lib
 
@@ -148,12 +151,18 @@ def attn_exact(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, rows=None, nthreads=0
 
 
 def attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, kv_order, block_n, n_sink,
-                 o_bf16=False, rows=None, nthreads=0, denom_mode=0):
+                 o_bf16=False, rows=None, nthreads=0, denom_mode=0, flip_slack=False):
     """FP8 pipeline emulation.  Returns (O [nrows, d] float32, collapse per row
     uint32, totals uint64[2] = {in sink-holding KV blocks, in other blocks}).
     Q, K: E4M3 bytes (uint8) or BF16 bit patterns (uint16, the kernel-faithful
     mode); V: E4M3 bytes.  denom_mode 0: l from the FP32 P, O = acc / (S l); 1: l from the cast values,
-    O = acc / l."""
+    O = acc / l.
+
+    flip_slack=True appends a fourth result, per row: how far O can move if each
+    cast whose fl32(S p) lies within a relative 2^-14 of an E4M3 rounding boundary
+    went to the neighbouring value (the sum over such casts of the E4M3 step times
+    max_k |v_jk|, rescaled like the accumulator, over the denominator; plus
+    step * max|O| per cast for the cast-value denominator); 0 for most rows."""
     for a in (Q8, K8, V8):
         assert a.flags.c_contiguous
     assert V8.dtype == np.uint8
@@ -162,13 +171,16 @@ def attn_emulate(Q8, K8, V8, B, H, Hkv, N, d, causal, scale, S, kv_order, block_
     O = np.empty((n_out, d), dtype=np.float32)
     cr = np.zeros(n_out, dtype=np.uint32)
     tot = np.zeros(2, dtype=np.uint64)
+    slack = np.zeros(n_out, dtype=np.float32) if flip_slack else None
     rc = lib().oracle_attn_emulate(_ptr(Q8), _ptr(K8), _ptr(V8), B, H, Hkv, N, d, int(causal),
                                    float(scale), float(S), int(kv_order), int(block_n),
                                    int(n_sink), int(bool(o_bf16)), _ptr(r), nr, _ptr(O),
                                    _ptr(cr), _ptr(tot), nthreads, int(denom_mode),
-                                   _qk_flag(Q8, K8))
+                                   _qk_flag(Q8, K8), _ptr(slack))
     if rc:
         raise ValueError("oracle_attn_emulate: bad shape")
+    if flip_slack:
+        return O, cr, tot, slack
     return O, cr, tot
 
 
@@ -184,6 +196,26 @@ def collapse_logits(logits, block_n, n_sink, S, kv_order, nthreads=0):
     if rc:
         raise ValueError("oracle_collapse_logits: bad shape")
     return cr, tot
+
+
+def attn_logits(logits, V8, rows_per_head, block_n, n_sink, S, kv_order, nthreads=0):
+    """The FP8 pipeline on given scaled logits [rows, N] with E4M3 values
+    V8 [heads, N, d] (row r reads head r // rows_per_head), non-causal.  Returns
+    (O_emu [rows, d] float32, O_exact [rows, d] float64, collapse per row)."""
+    x = np.ascontiguousarray(logits, dtype=np.float32)
+    V8 = np.ascontiguousarray(V8, dtype=np.uint8)
+    rows, N = x.shape
+    heads, Nv, d = V8.shape
+    assert Nv == N and heads * rows_per_head >= rows
+    Oe = np.empty((rows, d), dtype=np.float32)
+    Ox = np.empty((rows, d), dtype=np.float64)
+    cr = np.zeros(rows, dtype=np.uint32)
+    rc = lib().oracle_attn_logits(_ptr(x), _ptr(V8), rows, int(rows_per_head), N, d,
+                                  int(block_n), int(n_sink), float(S), int(kv_order), _ptr(Oe),
+                                  _ptr(Ox), _ptr(cr), nthreads)
+    if rc:
+        raise ValueError("oracle_attn_logits: bad shape")
+    return Oe, Ox, cr
 
 
 def collapse_denominator(B, H, N, n_sink, causal):

@@ -21,6 +21,9 @@
 //   * collapse_logits : the same online softmax on given scaled logits, used
 //                  for the closed-form underflow fraction F(Delta,S)
 //                  (Methodology, theoretical framework).
+//   * attn_logits : the pipeline on given scaled logits with a value matrix,
+//                  plus the float64 softmax of the same logits: the pages' MSE
+//                  experiments (Experimental results) in their own logit model.
 // All FP32 sums run left to right in the order stated at each loop.
 #include <cmath>
 #include <cstdint>
@@ -130,11 +133,12 @@ struct RowState {
 
 // One KV block of the FP8 pipeline for one row.
 //   s[j]  : scaled logits (FP32), -inf where masked
-//   on return: pt[j] = E4M3 code of fl32(S * p_j); alpha = rescale of the old state
+//   on return: pt[j] = E4M3 code of fl32(S * p_j); alpha = rescale of the old state;
+//   tv[j] = fl32(S * p_j) when tv is not NULL
 //   collapse counted for j_global >= n_sink with p_j > 0 and code magnitude 0.
 // Returns the number of collapsed entries.
 int softmax_block(const float* s, int n, int j0, int n_sink, float S, RowState& st,
-                  uint8_t* pt, float* alpha_out) {
+                  uint8_t* pt, float* alpha_out, float* tv = nullptr) {
     float mblk = kNegInf;
     for (int j = 0; j < n; ++j) mblk = std::fmax(mblk, s[j]);
     float m_new = std::fmax(st.m, mblk);
@@ -150,6 +154,7 @@ int softmax_block(const float* s, int n, int j0, int n_sink, float S, RowState& 
         float t = S * p;                          // fl32(S * p)
         uint8_t c = e4m3_encode(t);
         pt[j] = c;
+        if (tv) tv[j] = t;
         if (p > 0.0f && (c & 0x7F) == 0 && (j0 + j) >= n_sink) ++collapsed;
     }
     st.l = alpha * st.l + rowsum;
@@ -159,6 +164,31 @@ int softmax_block(const float* s, int n, int j0, int n_sink, float S, RowState& 
 }
 
 inline bool block_has_sink(int blk, int block_n, int n_sink) { return blk * block_n < n_sink; }
+
+// Exposure of one cast to a rounding flip.  The kernel's p differs from this
+// emulation's by a few FP32 ulps (its exponential and its QK^T summation
+// order), so a t = fl32(S * p) lying within a relative FLIP_TOL of an E4M3
+// rounding boundary (the midpoint between two adjacent E4M3 values, 2^-10
+// included) may be cast to the neighbouring value on the kernel's side.
+// Returns the E4M3 step such a flip would move dec(pt) by, 0 when t is not
+// that close to a boundary.
+const double FLIP_TOL = 0x1p-14;
+
+double flip_step(float t, uint8_t code) {
+    if (!(t > 0.0f)) return 0.0;
+    const int c = code & 0x7F;
+    const double v = e4m3_value((uint8_t)c);
+    double step = 0.0;
+    if (c < 0x7E) {                                    // boundary above (448 saturates)
+        const double up = e4m3_value((uint8_t)(c + 1));
+        if (std::fabs((double)t - 0.5 * (v + up)) <= FLIP_TOL * t) step = up - v;
+    }
+    if (c > 0) {                                       // boundary below
+        const double lo = e4m3_value((uint8_t)(c - 1));
+        if (std::fabs((double)t - 0.5 * (v + lo)) <= FLIP_TOL * t) step = std::max(step, v - lo);
+    }
+    return step;
+}
 
 }  // namespace
 
@@ -259,7 +289,7 @@ int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
                         int kv_order, int block_n, int n_sink, int o_bf16,
                         const int64_t* rows, int64_t nrows,
                         float* O, uint32_t* collapse_rows, uint64_t* collapse_totals,
-                        int nthreads, int denom_mode, int qk_bf16) {
+                        int nthreads, int denom_mode, int qk_bf16, float* flip_slack) {
     if (H % Hkv || block_n <= 0) return -1;
     Shape sh{B, H, Hkv, N, d};
     if (!rows) nrows = (int64_t)B * H * N;
@@ -270,7 +300,7 @@ int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
     uint64_t tot_sink = 0, tot_other = 0;
     #pragma omp parallel num_threads(nt) reduction(+ : tot_sink, tot_other)
     {
-        std::vector<float> q(d), acc(d), s(block_n), vdec((size_t)block_n * d);
+        std::vector<float> q(d), acc(d), s(block_n), tv(block_n), vdec((size_t)block_n * d);
         std::vector<uint8_t> pt(block_n);
         #pragma omp for schedule(dynamic, 4)
         for (int64_t t = 0; t < nrows; ++t) {
@@ -284,6 +314,8 @@ int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
             RowState st;
             float lq = 0.0f;   // denominator from the cast values (denom_mode 1)
             uint32_t row_collapse = 0;
+            // flip exposure, rescaled like acc: sum of step * max_k |v_jk| and of step
+            double sa = 0.0, sb = 0.0;
             const int last = causal ? i / block_n : nblocks - 1;
             for (int step = 0; step <= last; ++step) {
                 const int blk = (kv_order == 0) ? step : last - step;
@@ -298,8 +330,22 @@ int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
                     s[jj] = scale * dot;
                 }
                 float alpha;
-                int c = softmax_block(s.data(), nb, j0, n_sink, S, st, pt.data(), &alpha);
+                int c = softmax_block(s.data(), nb, j0, n_sink, S, st, pt.data(), &alpha,
+                                      flip_slack ? tv.data() : nullptr);
                 row_collapse += (uint32_t)c;
+                if (flip_slack) {
+                    sa *= alpha;
+                    sb *= alpha;
+                    for (int jj = 0; jj < nb; ++jj) {
+                        const double st_j = flip_step(tv[jj], pt[jj]);
+                        if (st_j == 0.0) continue;
+                        const uint8_t* vp = V + kvbase + (int64_t)(j0 + jj) * d;
+                        double vmax = 0.0;
+                        for (int k = 0; k < d; ++k) vmax = std::max(vmax, std::fabs(e4m3_value(vp[k])));
+                        sa += st_j * vmax;
+                        sb += st_j;
+                    }
+                }
                 if (block_has_sink(blk, block_n, n_sink)) tot_sink += (uint64_t)c;
                 else tot_other += (uint64_t)c;
                 float qsum = 0.0f;
@@ -314,16 +360,87 @@ int oracle_attn_emulate(const void* Q, const void* K, const uint8_t* V,
                 }
             }
             float denom = denom_mode ? lq : S * st.l;
+            double omax = 0.0;
             for (int k = 0; k < d; ++k) {
                 float o = acc[k] / denom;
                 O[t * d + k] = o_bf16 ? bf16_rne(o) : o;
+                omax = std::max(omax, std::fabs((double)o));
             }
+            // a flip moves the numerator by step * v_j and, with the cast-value
+            // denominator, the denominator by step as well
+            if (flip_slack)
+                flip_slack[t] = (float)((sa + (denom_mode ? sb * omax : 0.0)) / (double)denom);
             if (collapse_rows) collapse_rows[t] = row_collapse;
         }
     }
     if (collapse_totals) {
         collapse_totals[0] += tot_sink;
         collapse_totals[1] += tot_other;
+    }
+    return 0;
+}
+
+// ---- the FP8 pipeline on given scaled logits, with values -------------------
+// The pages' experiments (Experimental results: MSE of forward S = 1 against the
+// optimised configurations, S = 256 against S = 448, at N = 4096 and sink
+// strength Delta) are stated for their logit model, where the logits are drawn
+// directly: sinks Delta + N(0,1), the rest N(0,1).  This runs the same steps as
+// oracle_attn_emulate on such logits:
+//   logits [nrows, N] are the s_j (non-causal; -inf entries are masked keys);
+//   V: E4M3 bytes [nheads, N, d]; row r reads head r / rows_per_head.
+//   O_emu[r]   : the emulated FP32 output, O = acc / fl32(S * l)
+//   O_exact[r] : float64 sum_j softmax_j(s) dec(v_j)
+//   collapse_rows[r] (nullable): collapsed non-sink entries of row r.
+int oracle_attn_logits(const float* logits, const uint8_t* V, int64_t nrows, int rows_per_head,
+                       int N, int d, int block_n, int n_sink, float S, int kv_order,
+                       float* O_emu, double* O_exact, uint32_t* collapse_rows, int nthreads) {
+    if (block_n <= 0 || rows_per_head <= 0) return -1;
+    const int nt = nthreads > 0 ? nthreads : omp_get_num_procs();
+    const int nblocks = (N + block_n - 1) / block_n;
+    #pragma omp parallel num_threads(nt)
+    {
+        std::vector<float> acc(d);
+        std::vector<double> acc64(d);
+        std::vector<uint8_t> pt(block_n);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < nrows; ++r) {
+            const float* s = logits + r * (int64_t)N;
+            const uint8_t* vh = V + (r / rows_per_head) * (int64_t)N * d;
+            // emulation, block by block in the visiting order
+            RowState st;
+            uint32_t rc = 0;
+            for (int k = 0; k < d; ++k) acc[k] = 0.0f;
+            for (int step = 0; step < nblocks; ++step) {
+                const int blk = (kv_order == 0) ? step : nblocks - 1 - step;
+                const int j0 = blk * block_n;
+                const int nb = std::min(block_n, N - j0);
+                float alpha;
+                rc += (uint32_t)softmax_block(s + j0, nb, j0, n_sink, S, st, pt.data(), &alpha);
+                for (int k = 0; k < d; ++k) acc[k] = alpha * acc[k];
+                for (int jj = 0; jj < nb; ++jj) {
+                    const float pv = g_dec[pt[jj]];
+                    if (pv == 0.0f) continue;
+                    const uint8_t* vp = vh + (int64_t)(j0 + jj) * d;
+                    for (int k = 0; k < d; ++k) acc[k] += pv * g_dec[vp[k]];
+                }
+            }
+            const float denom = S * st.l;
+            for (int k = 0; k < d; ++k) O_emu[r * d + k] = acc[k] / denom;
+            if (collapse_rows) collapse_rows[r] = rc;
+            // float64 softmax of the same logits
+            double mx = -std::numeric_limits<double>::infinity();
+            for (int j = 0; j < N; ++j) mx = std::max(mx, (double)s[j]);
+            double sum = 0.0;
+            for (int k = 0; k < d; ++k) acc64[k] = 0.0;
+            for (int j = 0; j < N; ++j) {
+                if (s[j] == kNegInf) continue;
+                const double e = std::exp((double)s[j] - mx);
+                sum += e;
+                const uint8_t* vp = vh + (int64_t)j * d;
+                for (int k = 0; k < d; ++k) acc64[k] += e * e4m3_value(vp[k]);
+            }
+            for (int k = 0; k < d; ++k) O_exact[r * d + k] = acc64[k] / sum;
+        }
     }
     return 0;
 }

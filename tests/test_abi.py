@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_params_layout(lib):
     assert lib.fp8attn_params_sizeof() == ctypes.sizeof(Params)
-    assert lib.fp8attn_version() == 102
+    assert lib.fp8attn_version() == 103
 
 
 def test_status_strings(lib):
@@ -69,6 +69,7 @@ def base_params(**kw):
     (dict(O=FAKE + 8), EINVAL), (dict(K=FAKE + 1), EINVAL),
     (dict(collapse_rows=FAKE), EINVAL), (dict(collapse_ctr=FAKE + 4), EINVAL),
     (dict(debug_skip_kv_step=-1), EINVAL), (dict(debug_skip_kv_step=2), EINVAL),
+    (dict(timeout_ns=1), EINVAL), (dict(timeout_ns=999_999), EINVAL),
     (dict(denominator=2), EINVAL), (dict(denominator=1, S=0.001), EINVAL),
     (dict(qk_dtype=2), EINVAL),
     (dict(q_begin=64, q_end=256), EINVAL), (dict(q_begin=0, q_end=257), EINVAL),

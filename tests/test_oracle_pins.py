@@ -19,8 +19,12 @@ Pins:
   softmax-then-cast computed with library routines), Q = 0, V -> 2V, no sink,
   and a non-recurrent brute-force restatement on tiny inputs;
   O* against a numpy float64 softmax;
-* P-M: MSE orderings of the paper's Experimental results on the Delta/S sweep
-  workload (B=1, H=8, N=4096, d=128) at Delta = 7, on sampled rows.
+* P-M: the MSE claims of the paper's Experimental results in the paper's own
+  logit model (sink logits Delta + N(0,1), the rest N(0,1), N = 4096,
+  Delta = 7), through the pipeline on given logits, which is itself pinned to
+  the Q/K emulation bit for bit and to a numpy float64 softmax; on the
+  sink-construction workload the orderings only (its magnitudes differ, see
+  the reading with that test).
 """
 import json
 import math
@@ -324,6 +328,97 @@ def test_causal_collapse_denominator(oracle_mod):
         assert oracle_mod.collapse_denominator(1, 1, N, ns, False) == N * (N - ns)
 
 
+# ------------------------------------------------- pipeline on given logits ---
+def _fp32_logits(oracle_mod, Q8, K8, scale):
+    """s = fl32(scale * fl32(sum_k q_k k_k)) with the sum taken left to right in
+    FP32, element by element (numpy float32 ops, no fused multiply-add): the
+    logits the Q/K emulation forms internally.  Q8 [rows, d], K8 [N, d] bytes."""
+    tab = oracle_mod.e4m3_table().astype(np.float32)
+    q, k = tab[Q8], tab[K8]
+    acc = np.zeros((q.shape[0], k.shape[0]), dtype=np.float32)
+    for i in range(q.shape[1]):
+        acc = (acc + np.outer(q[:, i], k[:, i]).astype(np.float32)).astype(np.float32)
+    return (np.float32(scale) * acc).astype(np.float32)
+
+
+@pytest.mark.parametrize("N,d,block_n", [(256, 32, 64), (200, 16, 64), (128, 64, 128)])
+def test_logit_pipeline_equals_qk_emulation(oracle_mod, N, d, block_n):
+    """attn_logits on the logits the Q/K emulation forms gives that emulation's
+    O and per-row collapse counts bit for bit (non-causal, both orders, three S,
+    two heads sharing nothing)."""
+    B, H = 1, 2
+    W = workload.make_sink_workload(B, H, H, N, d, 4, 9.0, seed=90 + N)
+    Q8, K8, V8 = _cast_inputs(oracle_mod, W)
+    logits = np.concatenate([_fp32_logits(oracle_mod, Q8[0, h], K8[0, h], W.scale)
+                             for h in range(H)])
+    for S in (1.0, 256.0, 448.0):
+        for order in (0, 1):
+            Oe, cr, _ = oracle_mod.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, W.scale, S, order,
+                                                block_n, 4)
+            Ol, Ox, crl = oracle_mod.attn_logits(logits, V8[0], N, block_n, 4, S, order)
+            assert np.array_equal(Ol, Oe), (S, order)
+            assert np.array_equal(crl, cr), (S, order)
+            ref = oracle_mod.attn_exact(Q8, K8, V8, B, H, H, N, d, 0, W.scale)
+            assert np.abs(Ox - ref).max() < 1e-5      # logits rounded to FP32 vs float64 dots
+
+
+def test_logit_pipeline_exact_output_matches_numpy(oracle_mod):
+    """O_exact of attn_logits against a numpy float64 softmax of the same logits
+    times the decoded values, with masked (-inf) keys and rows spread over heads."""
+    rng = np.random.default_rng(4)
+    rows, N, d, heads = 12, 300, 16, 3
+    s = rng.standard_normal((rows, N)).astype(np.float32) * 3
+    s[:, 250:] = -np.inf
+    s[:, :4] += 6
+    V8 = oracle_mod.e4m3_encode(rng.standard_normal((heads, N, d)).astype(np.float32))
+    _, Ox, _ = oracle_mod.attn_logits(s, V8, rows // heads, 64, 4, 256.0, 1)
+    x = s.astype(np.float64)
+    P = np.exp(x - x.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    v = oracle_mod.e4m3_table()[V8]
+    ref = np.stack([P[r] @ v[r // (rows // heads)] for r in range(rows)])
+    assert np.abs(Ox - ref).max() < 1e-12
+
+
+def _pages_model_mse(oracle_mod, heads, rows_per_head, delta, seed, configs, N=4096, d=128):
+    """MSE against float64 attention, per (order, S), in the pages' logit model:
+    per row, sink logits delta + N(0,1) on the first 4 keys and N(0,1) on the
+    rest; each head its own E4M3 V ~ N(0,1), shared by its rows."""
+    rows = heads * rows_per_head
+    s = workload.ideal_logits(rows, N, 4, delta, seed)
+    V8 = np.empty((heads, N, d), dtype=np.uint8)
+    for h in range(heads):
+        V8[h] = oracle_mod.e4m3_encode(
+            workload.normals(seed, workload.STREAM_V, h * N * d, N * d).reshape(N, d))
+    mse = {}
+    for order, S in configs:
+        Oe, Ox, _ = oracle_mod.attn_logits(s, V8, rows_per_head, 128, 4, S, order)
+        mse[(order, S)] = float(np.mean((Oe.astype(np.float64) - Ox) ** 2))
+    return mse
+
+
+def test_mse_claims_in_the_pages_logit_model(oracle_mod):
+    """Experimental results, in the pages' own setting (N = 4096, Delta = 7,
+    four sinks at Delta + N(0,1), unit-variance non-sink logits), 128 heads of
+    32 rows, each head with its own values:
+    * forward S = 1 has 3-10x the MSE of the best optimised configuration (the
+      pages' band as printed);
+    * reverse + 256 is indistinguishable from forward + 256 (within 5%);
+    * forward S = 256 is below forward S = 448.  The pages put it about 10-15%
+      lower; in this model the expectation is about 8% lower, with a spread of
+      about +-0.015 per 4096-row sample, so the band is the pages' [0.85, 0.90]
+      widened by that spread and that offset: [0.82, 0.95]."""
+    mse = _pages_model_mse(oracle_mod, 128, 32, 7.0, workload.CONFIG_SEED_BASE + 7,
+                           [(0, 1.0), (0, 256.0), (0, 448.0), (1, 256.0), (1, 1.0)])
+    best = min(mse[(0, 256.0)], mse[(1, 256.0)], mse[(1, 1.0)])
+    g = GOLDEN["mse_ratio_forward_S1"]
+    assert g["lo"] <= mse[(0, 1.0)] / best <= g["hi"], mse
+    g = GOLDEN["mse_S256_vs_S448"]
+    r = mse[(0, 256.0)] / mse[(0, 448.0)]
+    assert 1 - g["hi"] - 0.03 <= r <= 1 - g["lo"] + 0.05, (r, mse)
+    assert abs(mse[(1, 256.0)] / mse[(0, 256.0)] - 1) < 0.05, mse
+
+
 # ------------------------------------------------------------------ P-M -------
 def test_mse_orderings_on_sweep_workload(oracle_mod):
     B, H, N, d, n_sink, block_n = 1, 8, 4096, 128, 4, 128
@@ -340,16 +435,14 @@ def test_mse_orderings_on_sweep_workload(oracle_mod):
             mse[(order, S)] = float(np.mean((O - ref) ** 2))
     base = mse[(0, 1.0)]
     best_fix = min(mse[(0, 256.0)], mse[(1, 256.0)], mse[(1, 1.0)])
-    # forward S = 1 is the worst configuration by a wide margin (paper: 3-10x;
-    # measured 2.7-2.8 at Delta = 7, 6.2-6.6 at Delta = 5 on 2048-row samples)
-    g = GOLDEN["mse_ratio_forward_S1"]
-    assert g["lo"] - 1.0 < base / best_fix < g["hi"], mse
-    assert base == max(mse.values())
-    # forward S = 256 beats forward S = 448 (paper: by about 10-15%; measured
-    # 4-12% over samples and Delta = 5, 7, 9; 384-row samples can flip it)
-    g = GOLDEN["mse_S256_vs_S448"]
-    assert 1 - g["hi"] - 0.05 < mse[(0, 256.0)] / mse[(0, 448.0)] < 0.97, mse
-    # one fix is enough: reverse + 256 ~ forward + 256 (saturation)
+    # The orderings hold on the sink construction too: forward S = 1 is the worst
+    # configuration, and one fix is enough (reverse + 256 ~ forward + 256).  Its
+    # magnitudes are smaller than the pages' (forward S = 1 at about 2.7x the
+    # best at Delta = 7): the construction's sink logits carry the query's
+    # projection on u and the keys' noise along u, so their spread is
+    # sqrt(1 + Delta^2 / 64 + 64 / d) rather than 1.  The pages' magnitudes are
+    # pinned in their own logit model (test_mse_claims_in_the_pages_logit_model).
+    assert base == max(mse.values()) and base / best_fix > 2.0, mse
     assert abs(mse[(1, 256.0)] / mse[(0, 256.0)] - 1) < 0.1, mse
 
 
@@ -444,9 +537,9 @@ def test_bf16_qk_exact_attention_matches_numpy(oracle_mod):
 
 
 def test_mse_orderings_kernel_faithful_mode(oracle_mod):
-    """The paper's Experimental results in its own setting (unquantised Q and
-    K, here BF16): forward S=1 3-10x worse, S=256 about 10-15% below S=448,
-    reverse+256 ~ forward+256 at Delta = 7, N = 4096."""
+    """The orderings of the paper's Experimental results with unquantised (BF16)
+    Q and K on the sink construction: forward S=1 the worst, reverse+256 ~
+    forward+256 at Delta = 7, N = 4096."""
     B, H, N, d = 1, 8, 4096, 128
     W = workload.make_sink_workload(B, H, H, N, d, 4, 7.0, seed=workload.CONFIG_SEED_BASE + 2)
     Q, K, V8 = _bf16_inputs(oracle_mod, W)
@@ -457,8 +550,40 @@ def test_mse_orderings_kernel_faithful_mode(oracle_mod):
         O, _, _ = oracle_mod.attn_emulate(Q, K, V8, B, H, H, N, d, 0, W.scale, S, order, 128, 4,
                                           rows=rows)
         mse[(order, S)] = float(np.mean((O - ref) ** 2))
-    # 2048 rows: a 10% MSE difference needs this many (384 rows can flip it)
+    # orderings only, as on the E4M3 sink construction (same logit spread)
     ratio = mse[(0, 1.0)] / min(mse[(0, 256.0)], mse[(1, 256.0)])
-    assert 2.0 < ratio < 10.5, mse                          # measured 2.6 (pages 3-10x)
-    assert 0.80 < mse[(0, 256.0)] / mse[(0, 448.0)] < 0.97, mse   # measured 0.94
+    assert mse[(0, 1.0)] == max(mse.values()) and ratio > 2.0, mse
     assert abs(mse[(1, 256.0)] / mse[(0, 256.0)] - 1) < 0.1, mse
+
+
+def test_flip_slack_special_cases(oracle_mod):
+    """The flip exposure reported with the emulation (used by the GPU parity
+    tolerance).  With Q = 0 every p is exactly 1 and fl32(S p) = S:
+    * S = 272, the midpoint between the E4M3 values 256 and 288 (ties to even:
+      cast to 256), and S within a relative 2^-16 of it: every key is exposed,
+      slack = 32 * sum_j max_k |v_jk| / (S * N);
+    * S = 272 (1 + 2^-12) and S = 264: no cast is within 2^-14 of a boundary,
+      slack = 0;
+    * the cast-value denominator adds 32 * max|O| per exposed key (over the
+      cast-value row sum, N times the cast of S)."""
+    B, H, N, d = 1, 1, 256, 32
+    W = workload.make_sink_workload(B, H, H, N, d, 0, 0.0, seed=95)
+    Q8 = np.zeros((B, H, N, d), dtype=np.uint8)
+    K8, V8 = oracle_mod.e4m3_encode(W.k), oracle_mod.e4m3_encode(W.v)
+    vmax = np.abs(oracle_mod.e4m3_table()[V8[0, 0]]).max(axis=1)
+    for S in (272.0, 272.0 * (1 + 2.0 ** -16)):
+        O, _, _, sl = oracle_mod.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, W.scale, S, 1, 64, 0,
+                                              flip_slack=True)
+        want = 32.0 * vmax.sum() / (np.float32(S) * np.float32(N))
+        assert np.allclose(sl, want, rtol=1e-6), (S, sl[:3], want)
+        O1, _, _, sl1 = oracle_mod.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, W.scale, S, 1, 64, 0,
+                                                denom_mode=1, flip_slack=True)
+        omax = np.abs(O1).max(axis=1)
+        # every p~ is the cast of S: 256 at the tie (to even), 288 just above it
+        l_cast = N * float(oracle_mod.e4m3_decode(oracle_mod.e4m3_encode(np.float32([S])))[0])
+        want1 = (32.0 * vmax.sum() + 32.0 * N * omax) / l_cast
+        assert np.allclose(sl1, want1, rtol=1e-5), (S, sl1[:3], want1[:3])
+    for S in (272.0 * (1 + 2.0 ** -12), 264.0):
+        _, _, _, sl = oracle_mod.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, W.scale, S, 1, 64, 0,
+                                              flip_slack=True)
+        assert not sl.any(), S
