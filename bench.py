@@ -139,9 +139,11 @@ def fp8_gemm_peak(dev, n=8192, reps=10):
 
 
 KERNEL_SOURCES = ["online_softmax_tcgen05_b200/csrc/fp8_attn_fwd.cu",
+                  "online_softmax_tcgen05_b200/csrc/fp8_attn_fwd_pair.cu",
                   "online_softmax_tcgen05_b200/csrc/attn_kernel.cuh",
                   "online_softmax_tcgen05_b200/csrc/sm100.cuh",
-                  "online_softmax_tcgen05_b200/csrc/exp2_poly.cuh"]
+                  "online_softmax_tcgen05_b200/csrc/exp2_poly.cuh",
+                  "online_softmax_tcgen05_b200/csrc/row_max.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_prefill_N32768.json")
 
 
@@ -635,6 +637,59 @@ def report_batched_orders(dev):
                           "TFLOP/s": round(flops / ms / 1e9, 1)}), flush=True)
 
 
+def report_schedules(dev, pairs=30):
+    """The two kernel schedules side by side in one process (fp8attn_set_schedule):
+    one query tile per CTA (default) and two query tiles per CTA with the softmax
+    warps taking turns on the exponential unit.  Prefill (causal GQA, reverse),
+    batched non-causal forward and reverse; counter on and off; 3 warm-up rounds
+    then `pairs` alternating timed launches of each schedule, median of each.
+    Both schedules' outputs and counters are compared bit for bit first."""
+    import torch
+    import workload
+    import online_softmax_tcgen05_b200 as fa
+    cases = [("prefill", (1, 32, 8, 32768, 128), 1, fa.KV_REVERSE, 8.0, 3),
+             ("batched forward", (4, 32, 32, 8192, 128), 0, fa.KV_FORWARD, 10.0, 4),
+             ("batched reverse", (4, 32, 32, 8192, 128), 0, fa.KV_REVERSE, 10.0, 4)]
+    scheds = [("one tile", fa.SCHEDULE_ONE_TILE), ("two tiles", fa.SCHEDULE_TWO_TILES)]
+    try:
+        for name, shape, causal, order, delta, cfg in cases:
+            W = workload.make_sink_workload(*shape, 4, delta, seed=workload.CONFIG_SEED_BASE + cfg)
+            ins = [fa.e4m3_cast(torch.from_numpy(x).to(dev)) for x in (W.q, W.k, W.v)]
+            del W
+            B, H, _, N, d = shape
+            flops = algorithmic_flops(B, H, N, d, bool(causal))
+            for count in (True, False):
+                runs = [(sn, sv, _ReportLaunch(fa, ins, shape, causal, 256.0, order, 4, count))
+                        for sn, sv in scheds]
+                if count:
+                    got = []
+                    for _, sv, r in runs:
+                        fa.set_schedule(sv)
+                        got.append((r.counts(), r.O.clone()))
+                    same = got[0][0] == got[1][0] and torch.equal(got[0][1], got[1][1])
+                times = {sn: [] for sn, _, _ in runs}
+                for i in range(3 + pairs):
+                    for sn, sv, r in runs:
+                        fa.set_schedule(sv)
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        r.launch()
+                        e1.record()
+                        torch.cuda.synchronize()
+                        if i >= 3:
+                            times[sn].append(e0.elapsed_time(e1))
+                for sn, _, _ in runs:
+                    ms = statistics.median(times[sn])
+                    print(json.dumps({"report": "schedules", "workload": name, "schedule": sn,
+                                      "counter": count, "median_ms": round(ms, 4),
+                                      "TFLOP/s": round(flops / ms / 1e9, 1),
+                                      "outputs_equal": same}), flush=True)
+            del ins
+    finally:
+        fa.set_schedule(fa.SCHEDULE_ONE_TILE)
+
+
 def report_e2e_timeline(dev, steps=2, warmup=4):
     """The prefill end to end through the host-buffer entry, profiled with CUPTI
     (torch.profiler) for diagnosis: per step, the time from the step's first
@@ -710,7 +765,8 @@ def main():
                          "the long-context problem split by kv heads (strong scaling)")
     ap.add_argument("--mode", choices=["full", "kernel"], default="full",
                     help="kernel: only the device-timed kernel loop (for profiling)")
-    ap.add_argument("--report", choices=["collapse", "configs", "batched-orders", "e2e-timeline"],
+    ap.add_argument("--report", choices=["collapse", "configs", "batched-orders", "e2e-timeline",
+                                         "schedules"],
                     default=None,
                     help="one GPU: JSON lines for the Delta/S collapse sweep against the closed "
                          "form, or the timing protocols of the larger configurations")
@@ -721,7 +777,7 @@ def main():
         torch.cuda.set_device(dev)
         {"collapse": report_collapse, "configs": report_configs,
          "batched-orders": report_batched_orders,
-         "e2e-timeline": report_e2e_timeline}[args.report](dev)
+         "e2e-timeline": report_e2e_timeline, "schedules": report_schedules}[args.report](dev)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -242,6 +242,21 @@ int fp8_attn_fwd_host(const fp8attn_params* p, fp8attn_host_plan* plan, void* wo
 
 int fp8_attn_fwd_host_noalloc(const fp8attn_params* p, fp8attn_stream_t stream);
 
+/* Kernel schedule of the device-buffer entries (and of the host-buffer entries,
+ * which call them).  Both compute the same operation, in the same order per
+ * row and with the same results:
+ *   FP8ATTN_SCHEDULE_ONE_TILE   one 128-row query tile per CTA, two CTAs per SM,
+ *                               whose softmax phases overlap by chance (default);
+ *   FP8ATTN_SCHEDULE_TWO_TILES  two query tiles per CTA that share one K/V
+ *                               stream (two heads of one kv head, or two
+ *                               consecutive tiles), one CTA per SM, the two
+ *                               tiles' softmax warps on each SM sub-partition
+ *                               taking turns on the exponential unit.
+ * Process-wide; returns the previous schedule, or FP8ATTN_EINVAL for an unknown
+ * value (nothing changed).  Calls already enqueued keep their schedule. */
+enum { FP8ATTN_SCHEDULE_ONE_TILE = 0, FP8ATTN_SCHEDULE_TWO_TILES = 1 };
+int fp8attn_set_schedule(int schedule);
+
 /* Human-readable name of a status code (static string). */
 const char* fp8attn_status_string(int status);
 

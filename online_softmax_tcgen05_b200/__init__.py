@@ -18,7 +18,8 @@ import math
 from dataclasses import dataclass
 
 from ._binding import (DENOM_CAST_P, DENOM_FP32_P, ECUDA, EINVAL, ETIMEOUT, EUNSUPPORTED,
-                       KV_FORWARD, KV_REVERSE, O_BF16, O_F32, OK, QK_BF16, QK_E4M3, Fp8AttnError,
+                       KV_FORWARD, KV_REVERSE, O_BF16, O_F32, OK, QK_BF16, QK_E4M3,
+                       SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES, Fp8AttnError, set_schedule,
                        HostPlan, device_status_string, fp8_attn_fwd, fp8_attn_fwd_ex,
                        fp8_attn_fwd_host, fp8_attn_fwd_host_noalloc, fp8_e4m3_scale_cast,
                        host_workspace_bytes, last_error, load_library, status_string)
@@ -28,7 +29,8 @@ __all__ = ["attention", "AttentionStats", "fp8_attn_fwd", "fp8_attn_fwd_ex",
            "fp8_e4m3_scale_cast", "load_library", "status_string", "last_error",
            "device_status_string", "Fp8AttnError", "KV_FORWARD", "KV_REVERSE", "O_BF16",
            "O_F32", "OK", "EINVAL", "EUNSUPPORTED", "ECUDA", "ETIMEOUT", "e4m3_cast",
-           "DENOM_FP32_P", "DENOM_CAST_P", "QK_E4M3", "QK_BF16"]
+           "DENOM_FP32_P", "DENOM_CAST_P", "QK_E4M3", "QK_BF16", "set_schedule",
+           "SCHEDULE_ONE_TILE", "SCHEDULE_TWO_TILES"]
 
 
 @dataclass

@@ -13,6 +13,7 @@ import math
 from . import _build
 
 KV_FORWARD, KV_REVERSE = 0, 1
+SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES = 0, 1
 O_BF16, O_F32 = 0, 1
 DENOM_FP32_P, DENOM_CAST_P = 0, 1
 QK_E4M3, QK_BF16 = 0, 1
@@ -59,6 +60,7 @@ SIGNATURES = {
     "fp8_attn_fwd_host": ([ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_void_p,
                            ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p], ctypes.c_int),
     "fp8_attn_fwd_host_noalloc": ([ctypes.POINTER(Params), ctypes.c_void_p], ctypes.c_int),
+    "fp8attn_set_schedule": ([ctypes.c_int], ctypes.c_int),
 }
 
 _lib = None
@@ -213,3 +215,12 @@ def fp8_attn_fwd_host_noalloc(Q, K, V, O, *, stream=None, **kw):
     p = _params(Q, K, V, O, **kw)
     _check(load_library().fp8_attn_fwd_host_noalloc(ctypes.byref(p), _stream(stream)),
            "fp8_attn_fwd_host_noalloc")
+
+
+def set_schedule(schedule: int) -> int:
+    """Select the kernel schedule (SCHEDULE_ONE_TILE or SCHEDULE_TWO_TILES) for
+    later calls, process-wide; returns the previous one."""
+    prev = load_library().fp8attn_set_schedule(int(schedule))
+    if prev < 0:
+        _check(prev, "fp8attn_set_schedule")
+    return prev

@@ -40,6 +40,7 @@
 #include "attn_kernel.cuh"
 #include "exp2_poly.cuh"
 #include "fp8attn.h"
+#include "row_max.cuh"
 #include "sm100.cuh"
 
 namespace fp8attn {
@@ -343,22 +344,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               if (j0 + j > lim) s[j] = -INFINITY;
           }
         }
-        // row max: 16 independent chains of three-input max, then a tree
-        float mx16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx16[i] = s[i];
-#pragma unroll
-        for (int j = 16; j + 16 < BN; j += 32)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
-        if constexpr ((BN - 16) % 32 != 0) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
-        }
-        float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
-                         fmax3(mx16[6], mx16[7], mx16[8]));
-        mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
-        mx = fmaxf(mx, mx16[15]);
+        const float mx = row_max<BN>(s);
         m_new = fmaxf(m_run, mx * c);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);

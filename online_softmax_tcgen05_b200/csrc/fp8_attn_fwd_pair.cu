@@ -46,7 +46,9 @@
 #include <cstdint>
 
 #include "attn_kernel.cuh"
+#include "exp2_poly.cuh"
 #include "fp8attn.h"
+#include "row_max.cuh"
 #include "sm100.cuh"
 
 namespace fp8attn {
@@ -65,7 +67,7 @@ struct Smem {
   // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], per tile: s_full,
   // s_free, p_full, o_done; drain
   static constexpr int NBAR = 1 + 4 * NSTAGE + 8 + 1;
-  static constexpr int MISC = BAR + 8 * NBAR;   // tmem slot, abort flag, never flag
+  static constexpr int MISC = BAR + 8 * NBAR;   // tmem slot, abort, never, MMA idle flags
   static constexpr int BYTES = MISC + 16;
   // at least 120 KB: one CTA per SM (the CTA takes all 512 TMEM columns)
   static constexpr int ALLOC = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
@@ -85,6 +87,36 @@ __device__ __forceinline__ int kv_block_at(int t, int T, int order) {
 // Named barriers of the exponential turns: SMSP k uses TURN_A + k (tile A may
 // start) and TURN_B + k (tile B may start); two warps (64 threads) each.
 constexpr uint32_t TURN_A = 1, TURN_B = 5;
+// What a turn covers: 1 = the exponentials and row sums; 2 = those, the E4M3
+// cast and the collapse count; 0 = no turns (the two tiles run freely).
+#ifndef FP8ATTN_TURN_SCOPE
+#define FP8ATTN_TURN_SCOPE 1
+#endif
+constexpr int TURN_SCOPE = FP8ATTN_TURN_SCOPE;
+#ifndef FP8ATTN_EXP_SPLIT
+#define FP8ATTN_EXP_SPLIT 0
+#endif
+constexpr bool EXP_SPLIT = FP8ATTN_EXP_SPLIT != 0;
+// Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
+// (exp2_poly.cuh) and the rest on MUFU ex2 during a warp's turn, when the FMA
+// pipe is otherwise nearly idle.
+#ifndef FP8ATTN_PAIR_POLY_OF_8
+#define FP8ATTN_PAIR_POLY_OF_8 0
+#endif
+constexpr int PAIR_POLY_OF_8 = FP8ATTN_PAIR_POLY_OF_8;
+
+// Waits of this kernel's roles: with a suspend-time hint (ns) a waiting warp
+// sleeps between probes instead of issuing them back to back.
+#ifndef FP8ATTN_PAIR_WAIT_HINT_NS
+#define FP8ATTN_PAIR_WAIT_HINT_NS 0
+#endif
+__device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
+                                      uint32_t where) {
+  if constexpr (FP8ATTN_PAIR_WAIT_HINT_NS > 0)
+    return mbar_wait_hint(bar, parity, ctl, where, FP8ATTN_PAIR_WAIT_HINT_NS);
+  else
+    return mbar_wait(bar, parity, ctl, where);
+}
 
 // The turns order execution, not memory (no memory clobber: the scores stay in
 // registers across them).  The running max passes through the wait and the row
@@ -125,6 +157,8 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 4);
   volatile uint32_t* never_flag = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 8);
+  // raised by the MMA warp once every MMA it issued has completed
+  volatile uint32_t* mma_idle = reinterpret_cast<volatile uint32_t*>(smem + L::MISC + 12);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Work unit: a row unit (a tile pair, or one tile for head pairs) of a plane
@@ -170,6 +204,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     *never_flag = 0;
+    *mma_idle = 0;
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -205,7 +240,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
       int k_issued = 0, v_issued = 0;
       auto load_k = [&](int t) -> bool {
         const int st = t % NSTAGE, n = t / NSTAGE;
-        if (t >= NSTAGE && !mbar_wait(bar_k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+        if (t >= NSTAGE && !pwait(bar_k_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
           return false;
         if (t + 1 == p.debug_skip_kv_step) return true;   // testing: leave this K tile out
         mbar_arrive_expect_tx(bar_k_full(st), BN * D * QB);
@@ -225,7 +260,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
       for (int t = 0; ok && t < T; ++t) {
         if (t + 1 < T && !load_k(t + 1)) break;
         const int st = t % NSTAGE, n = t / NSTAGE;
-        if (t >= NSTAGE && !mbar_wait(bar_v_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
+        if (t >= NSTAGE && !pwait(bar_v_empty(st), (n - 1) & 1, ctl, WAIT_PROD_KV_EMPTY))
           break;
         mbar_arrive_expect_tx(bar_v_full(st), BN * D);
         tma_load_3d(sV + st * BN * D, &tmV, bar_v_full(st), 0, kv_block_at(t, T, p.kv_order) * BN,
@@ -250,7 +285,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
     constexpr uint32_t SWZ_P = (BN == 128) ? SWZ_128B : SWZ_64B;
     constexpr uint32_t IDESC_QK = idesc_e4m3_f32(BM, BN, 0, 0);
     constexpr uint32_t IDESC_PV = idesc_e4m3_f32(BM, D, 0, 1);
-    bool ok = mbar_wait(bar_q_full, 0, ctl, WAIT_MMA_Q);
+    bool ok = pwait(bar_q_full, 0, ctl, WAIT_MMA_Q);
     auto issue_qk = [&](int x, int st) {
       tc_fence_after();
       if (lane == 0) {
@@ -293,43 +328,56 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       __syncwarp();
     };
-    if (ok) ok = mbar_wait(bar_k_full(0), 0, ctl, WAIT_MMA_K);
+    if (ok) ok = pwait(bar_k_full(0), 0, ctl, WAIT_MMA_K);
     if (ok) {
       issue_qk(0, 0);
       issue_qk(1, 0);
       if (lane == 0) mma_commit(bar_k_empty(0));
       __syncwarp();
     }
+    // Issue order per step t, the order in which the turns make the operands
+    // ready (tile B runs about half a block behind tile A): QK^T_A(t+1),
+    // P~V_B(t-1), QK^T_B(t+1), P~V_A(t).  Each tile's S(t+1) commit still
+    // follows its own P~V(t-1).
+    auto pv_b = [&](int t) -> bool {   // P~V_B(t), then V stage t is free
+      const int st = t % NSTAGE;
+      if (!pwait(bar_p_full(1), t & 1, ctl, WAIT_MMA_P)) return false;
+      issue_pv(1, st, t);
+      if (lane == 0) mma_commit(bar_v_empty(st));
+      __syncwarp();
+      return true;
+    };
     for (int t = 0; ok && t < T; ++t) {
+      const int st1 = (t + 1) % NSTAGE, ph1 = ((t + 1) / NSTAGE) & 1;
       if (t + 1 < T) {
-        const int st1 = (t + 1) % NSTAGE, ph1 = ((t + 1) / NSTAGE) & 1;
-        ok = mbar_wait(bar_k_full(st1), ph1, ctl, WAIT_MMA_K) &&
-             mbar_wait(bar_s_free(0), t & 1, ctl, WAIT_MMA_S_FREE);
+        ok = pwait(bar_k_full(st1), ph1, ctl, WAIT_MMA_K) &&
+             pwait(bar_s_free(0), t & 1, ctl, WAIT_MMA_S_FREE);
         if (!ok) break;
         issue_qk(0, st1);
-        ok = mbar_wait(bar_s_free(1), t & 1, ctl, WAIT_MMA_S_FREE);
+      }
+      if (t > 0 && !(ok = pv_b(t - 1))) break;
+      if (t + 1 < T) {
+        ok = pwait(bar_s_free(1), t & 1, ctl, WAIT_MMA_S_FREE);
         if (!ok) break;
         issue_qk(1, st1);
         if (lane == 0) mma_commit(bar_k_empty(st1));
         __syncwarp();
       }
       const int st = t % NSTAGE, ph = (t / NSTAGE) & 1;
-      ok = mbar_wait(bar_v_full(st), ph, ctl, WAIT_MMA_V) &&
-           mbar_wait(bar_p_full(0), t & 1, ctl, WAIT_MMA_P);
+      ok = pwait(bar_v_full(st), ph, ctl, WAIT_MMA_V) &&
+           pwait(bar_p_full(0), t & 1, ctl, WAIT_MMA_P);
       if (!ok) break;
       issue_pv(0, st, t);
-      ok = mbar_wait(bar_p_full(1), t & 1, ctl, WAIT_MMA_P);
-      if (!ok) break;
-      issue_pv(1, st, t);
-      if (lane == 0) mma_commit(bar_v_empty(st));
-      __syncwarp();
     }
-    if (!ok) {
-      // drain every MMA this warp issued before TMEM is released
+    if (ok) ok = pv_b(T - 1);
+    {
+      // wait for every MMA this warp issued (after an abort too), then tell an
+      // aborting softmax warp that TMEM and the P~ tiles are no longer in use
       const WaitCtl drain{never_flag, DRAIN_TIMEOUT_NS};
       if (lane == 0) mma_commit(bar_drain);
       __syncwarp();
       mbar_wait(bar_drain, 0, drain, 0);
+      if (lane == 0) *mma_idle = 1;
     }
   } else {
     // ------------------------------------------------------------- softmax --
@@ -355,9 +403,21 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
     // Tile A takes the first exponential turn.  Every block runs the same code
     // whether or not the CTA is aborting (only the waits are skipped then, and
     // the results are not stored), so both warps of an SMSP always take the
-    // same number of turns.
-    if (x == 1) turn_pass(other_turn, 0.f);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(x), 0, ctl, WAIT_SM_S_FULL));
+    // same number of turns.  An aborting warp first waits (bounded) until the
+    // MMA warp has drained, so that its later TMEM and P~ accesses race with
+    // no MMA in flight.
+    bool settled = false;
+    auto settle = [&](bool ok_now) {
+      if (!ok_now && !settled) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!*mma_idle && globaltimer_ns() - t0 < 2 * DRAIN_TIMEOUT_NS) {
+        }
+        settled = true;
+      }
+    };
+    if (TURN_SCOPE && x == 1) turn_pass(other_turn, 0.f);
+    bool ok = __all_sync(0xffffffffu, pwait(bar_s_full(x), 0, ctl, WAIT_SM_S_FULL));
+    settle(ok);
     for (int t = 0; t < T; ++t) {
       const int j0 = kv_block_at(t, T, p.kv_order) * BN;
       uint32_t sr[BN];
@@ -380,140 +440,149 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
           for (int j = 0; j < BN; ++j)
             if (j0 + j > lim) s[j] = -INFINITY;
         }
-        // row max: 16 independent chains of three-input max, then a tree
-        float mx16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx16[i] = s[i];
-#pragma unroll
-        for (int j = 16; j + 16 < BN; j += 32)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx16[i] = fmax3(mx16[i], s[j + i], s[j + 16 + i]);
-        if constexpr ((BN - 16) % 32 != 0) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], s[BN - 16 + i]);
-        }
-        float mx = fmax3(fmax3(mx16[0], mx16[1], mx16[2]), fmax3(mx16[3], mx16[4], mx16[5]),
-                         fmax3(mx16[6], mx16[7], mx16[8]));
-        mx = fmax3(mx, fmax3(mx16[9], mx16[10], mx16[11]), fmax3(mx16[12], mx16[13], mx16[14]));
-        mx = fmaxf(mx, mx16[15]);
+        const float mx = row_max<BN>(s);
         m_new = fmaxf(m_run, mx * c);
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
       }
 
-      // ---- this SMSP's exponential turn: 2^(s*c - m + log2S) and row sums
-      const float m_turn = turn_wait(my_turn, m_new);
-      float rowsum;
-      {
+      // ---- this SMSP's turn on the exponential unit ----
+      // 2^(s*c - m + log2S) with its row sums, then the E4M3 cast and the
+      // collapse count, as one body (branch-free on plain blocks) so that the
+      // integer work fills the issue slots between the exponentials.
+      const float m_turn = TURN_SCOPE ? turn_wait(my_turn, m_new) : m_new;
+      auto block_body = [&](auto plain_tag) {
+        constexpr bool PLAIN = decltype(plain_tag)::value;
         const float m_use = (m_turn == -INFINITY) ? 0.f : m_turn;
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
         float2 acc8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
+        if constexpr (EXP_SPLIT) {
+          // one warp alone on the unit: issue every ex2 first and add the row
+          // sums afterwards, so that no sum waits on an ex2 still in flight
 #pragma unroll
-        for (int q = 0; q < BN / 2; ++q) {
-          const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
-          s[2 * q] = ex2_approx(y.x);
-          s[2 * q + 1] = ex2_approx(y.y);
-          acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
+          for (int q = 0; q < BN / 2; ++q) {
+            const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
+            s[2 * q] = ex2_approx(y.x);
+            s[2 * q + 1] = ex2_approx(y.y);
+          }
+#pragma unroll
+          for (int q = 0; q < BN / 2; ++q)
+            acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < BN / 2; ++q) {
+            const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
+            if ((q & 7) < PAIR_POLY_OF_8) {
+              const float2 e = exp2_poly2(y);
+              s[2 * q] = e.x;
+              s[2 * q + 1] = e.y;
+            } else {
+              s[2 * q] = ex2_approx(y.x);
+              s[2 * q + 1] = ex2_approx(y.y);
+            }
+            acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
+          }
         }
 #pragma unroll
         for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
           for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
-        rowsum = acc8[0].x + acc8[0].y;
-      }
-      // hand the unit to the other tile's warp (tile B's last block has no
-      // taker: tile A is done with its turns)
-      if (x == 0 || t + 1 < T) turn_pass(other_turn, rowsum);
-
-      {
-        if (!p.denom_cast) l = alpha * l + rowsum;
+        const float rowsum = acc8[0].x + acc8[0].y;
+        if constexpr (TURN_SCOPE == 1) {
+          if (x == 0 || t + 1 < T) turn_pass(other_turn, rowsum);
+        }
+        if (PLAIN || !p.denom_cast) l = alpha * l + rowsum;
         // the E4M3 cast of S*p, four keys per word; off the plain path fl(s_mul * x):
         // the FP32 product S*p when S is not a power of two, an exact multiply by
         // 1 when S*p came out of the exponential
-        auto cast_count = [&](auto plain_tag) {
-          constexpr bool PLAIN = decltype(plain_tag)::value;
-          const float2 sm2 = make_float2(p.s_mul, p.s_mul);
+        const float2 sm2 = make_float2(p.s_mul, p.s_mul);
 #pragma unroll
-          for (int q = 0; q < BN / 4; ++q) {
-            if constexpr (PLAIN) {
-              pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-            } else {
-              const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), sm2);
-              const float2 b = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), sm2);
-              pw[q] = pack_e4m3x4(a.x, a.y, b.x, b.y);
-            }
+        for (int q = 0; q < BN / 4; ++q) {
+          if constexpr (PLAIN) {
+            pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+          } else {
+            const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), sm2);
+            const float2 b = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), sm2);
+            pw[q] = pack_e4m3x4(a.x, a.y, b.x, b.y);
           }
+        }
+        if constexpr (!PLAIN) {
+          if (p.denom_cast) {
+            // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32
+            // bit 20 form a float 2^-120 times the E4M3 value (subnormals too)
+            float2 d4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q) {
+              const uint32_t w = pw[q];
+              const float2 lo = make_float2(__uint_as_float((w & 0x7Fu) << 20),
+                                            __uint_as_float((w & 0x7F00u) << 12));
+              const float2 hi = make_float2(__uint_as_float((w & 0x7F0000u) << 4),
+                                            __uint_as_float((w & 0x7F000000u) >> 4));
+              d4[q & 3] = __fadd2_rn(d4[q & 3], __fadd2_rn(lo, hi));
+            }
+            d4[0] = __fadd2_rn(__fadd2_rn(d4[0], d4[1]), __fadd2_rn(d4[2], d4[3]));
+            l = alpha * l + (d4[0].x + d4[0].y) * 0x1p120f;
+          }
+        }
+        if constexpr (COUNT) {
+          // Collapse: a visible non-sink key whose E4M3 byte is zero (P~ is never
+          // negative, so byte 0 <=> the cast flushed S*p to zero)
+          uint32_t cblk;
+          if (PLAIN || (j0 >= p.n_sink && !need_mask)) {
+            // bytes are 0x00..0x7F, so w + 0x7F7F7F7F sets bit 7 of exactly the
+            // nonzero bytes without carries; dp4a sums those flags (x128)
+            uint32_t nz4[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q)
+              nz4[q & 3] = __dp4a((pw[q] + 0x7F7F7F7Fu) & 0x80808080u, 0x01010101u, nz4[q & 3]);
+            cblk = BN - (((nz4[0] + nz4[1]) + (nz4[2] + nz4[3])) >> 7);
+          } else {
+            // blocks holding a sink or a masked key count the lanes with
+            // n_sink <= j <= last visible key only
+            uint32_t zacc = 0;
+            const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q) {
+              const uint32_t w = pw[q];
+              uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
+              const int a = lo - 4 * q, bq = hi - 4 * q;
+              const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
+              const uint32_t mhi =
+                  bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
+              zacc += (y & mlo & mhi) >> 7;
+            }
+            cblk = (zacc * 0x01010101u) >> 24;
+          }
+          cnt += cblk;
           if constexpr (!PLAIN) {
-            if (p.denom_cast) {
-              // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32
-              // bit 20 form a float 2^-120 times the E4M3 value (subnormals too)
-              float2 d4[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) d4[i] = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int q = 0; q < BN / 4; ++q) {
-                const uint32_t w = pw[q];
-                const float2 lo = make_float2(__uint_as_float((w & 0x7Fu) << 20),
-                                              __uint_as_float((w & 0x7F00u) << 12));
-                const float2 hi = make_float2(__uint_as_float((w & 0x7F0000u) << 4),
-                                              __uint_as_float((w & 0x7F000000u) >> 4));
-                d4[q & 3] = __fadd2_rn(d4[q & 3], __fadd2_rn(lo, hi));
-              }
-              d4[0] = __fadd2_rn(__fadd2_rn(d4[0], d4[1]), __fadd2_rn(d4[2], d4[3]));
-              l = alpha * l + (d4[0].x + d4[0].y) * 0x1p120f;
-            }
+            if (j0 < p.n_sink) cnt_sink += cblk;
           }
-          if constexpr (COUNT) {
-            // Collapse: a visible non-sink key whose E4M3 byte is zero (P~ is never
-            // negative, so byte 0 <=> the cast flushed S*p to zero)
-            uint32_t cblk;
-            if (PLAIN || (j0 >= p.n_sink && !need_mask)) {
-              // bytes are 0x00..0x7F, so w + 0x7F7F7F7F sets bit 7 of exactly the
-              // nonzero bytes without carries; dp4a sums those flags (x128)
-              uint32_t nz4[4] = {0, 0, 0, 0};
-#pragma unroll
-              for (int q = 0; q < BN / 4; ++q)
-                nz4[q & 3] = __dp4a((pw[q] + 0x7F7F7F7Fu) & 0x80808080u, 0x01010101u, nz4[q & 3]);
-              cblk = BN - (((nz4[0] + nz4[1]) + (nz4[2] + nz4[3])) >> 7);
-            } else {
-              // blocks holding a sink or a masked key count the lanes with
-              // n_sink <= j <= last visible key only
-              uint32_t zacc = 0;
-              const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);
-#pragma unroll
-              for (int q = 0; q < BN / 4; ++q) {
-                const uint32_t w = pw[q];
-                uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
-                const int a = lo - 4 * q, bq = hi - 4 * q;
-                const uint32_t mlo =
-                    a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
-                const uint32_t mhi =
-                    bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
-                zacc += (y & mlo & mhi) >> 7;
-              }
-              cblk = (zacc * 0x01010101u) >> 24;
-            }
-            cnt += cblk;
-            if constexpr (!PLAIN) {
-              if (j0 < p.n_sink) cnt_sink += cblk;
-            }
-          }
-        };
+        }
+        if constexpr (TURN_SCOPE == 2) {
+          // hand the unit to the other tile's warp (tile B's last block has no
+          // taker: tile A is done with its turns)
+          if (x == 0 || t + 1 < T) turn_pass(other_turn, __uint_as_float(pw[BN / 4 - 1]));
+        }
+      };
+      {
         if (plain)
-          cast_count(BoolTag<true>{});
+          block_body(BoolTag<true>{});
         else
-          cast_count(BoolTag<false>{});
+          block_body(BoolTag<false>{});
         // P~V(t-1) must be done before the P~ tile is rewritten and O rescaled.
         // The commit that completes S(t+1) tracks every MMA issued before
         // QK^T(t+1), P~V(t-1) among them; the last block waits for P~V(t-1).
         if (t + 1 < T) {
           ok = ok && __all_sync(0xffffffffu,
-                                mbar_wait(bar_s_full(x), (t + 1) & 1, ctl, WAIT_SM_S_FULL));
+                                pwait(bar_s_full(x), (t + 1) & 1, ctl, WAIT_SM_S_FULL));
         } else if (t > 0) {
           ok = ok && __all_sync(0xffffffffu,
-                                mbar_wait(bar_o_done(x), (t - 1) & 1, ctl, WAIT_SM_O_DONE));
+                                pwait(bar_o_done(x), (t - 1) & 1, ctl, WAIT_SM_O_DONE));
         }
+        settle(ok);
       }
       {
         tc_fence_after();
@@ -560,7 +629,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
 
     if (ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(x), (T - 1) & 1, ctl, WAIT_EPI_O_DONE));
+      ok = __all_sync(0xffffffffu, pwait(bar_o_done(x), (T - 1) & 1, ctl, WAIT_EPI_O_DONE));
     }
     if (ok) {
       tc_fence_after();

@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -15,11 +16,10 @@
 #include "attn_kernel.cuh"
 #include "fp8attn.h"
 
-// 1: the two-tile kernel (fp8_attn_fwd_pair.cu); 0: one tile per CTA
-// (fp8_attn_fwd.cu).  Same arithmetic, different schedule.
-#ifndef FP8ATTN_PAIR_KERNEL
-#define FP8ATTN_PAIR_KERNEL 0
-#endif
+namespace {
+// fp8attn_set_schedule: the kernel that fp8_attn_fwd_ex launches
+std::atomic<int> g_schedule{FP8ATTN_SCHEDULE_ONE_TILE};
+}  // namespace
 
 namespace fp8attn {
 
@@ -143,7 +143,7 @@ bool make_map(CUtensorMap* m, const void* base, int d, int rows, int planes, int
 
 extern "C" {
 
-int fp8attn_version(void) { return 103; }
+int fp8attn_version(void) { return 104; }
 
 size_t fp8attn_params_sizeof(void) { return sizeof(fp8attn_params); }
 
@@ -159,6 +159,13 @@ const char* fp8attn_status_string(int status) {
 }
 
 const char* fp8attn_last_error(void) { return fp8attn::last_error(); }
+
+int fp8attn_set_schedule(int schedule) {
+  fp8attn::clear_error();
+  if (schedule != FP8ATTN_SCHEDULE_ONE_TILE && schedule != FP8ATTN_SCHEDULE_TWO_TILES)
+    return fail(FP8ATTN_EINVAL, "schedule must be FP8ATTN_SCHEDULE_ONE_TILE or _TWO_TILES");
+  return g_schedule.exchange(schedule);
+}
 
 const char* fp8attn_device_status_string(unsigned int word) {
   if (word == 0) return "";
@@ -213,7 +220,7 @@ int fp8_attn_fwd_ex(const fp8attn_params* p, fp8attn_stream_t stream) {
   // otherwise two consecutive tiles of one head; its scheduling groups count
   // plane units (head pairs or planes)
   kp.pair_heads = (kp.group % 2 == 0) ? 1 : 0;
-  const bool use_pair = FP8ATTN_PAIR_KERNEL != 0;
+  const bool use_pair = g_schedule.load(std::memory_order_relaxed) == FP8ATTN_SCHEDULE_TWO_TILES;
   if (use_pair && kp.pair_heads) kp.sched_group /= 2;
   kp.causal = p->causal;
   kp.kv_order = p->kv_order;

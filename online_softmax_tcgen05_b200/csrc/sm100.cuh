@@ -49,6 +49,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete may be suspended
+// until it completes or `hint_ns` nanoseconds pass (the suspend-time hint of
+// try_wait), instead of returning at once: a waiting warp then issues few
+// probes, leaving the SMSP's memory-instruction queue to the other warps.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared state of the bounded waits of one CTA.  A wait that runs past the
 // time limit raises `abort` so that every other role leaves its loop too.
 struct WaitCtl {
@@ -66,6 +83,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (*ctl.abort) return false;
+    if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+      atomicCAS(const_cast<uint32_t*>(ctl.abort), 0u, where);
+      return false;
+    }
+  }
+}
+
+// mbar_wait whose probes may suspend the thread for up to hint_ns each (see
+// mbar_try_wait_hint); the same time bound and abort rules.
+__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, const WaitCtl& ctl,
+                                               uint32_t where, uint32_t hint_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
     if (*ctl.abort) return false;
     if (globaltimer_ns() - t0 > ctl.timeout_ns) {
       atomicCAS(const_cast<uint32_t*>(ctl.abort), 0u, where);

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_params_layout(lib):
     assert lib.fp8attn_params_sizeof() == ctypes.sizeof(Params)
-    assert lib.fp8attn_version() == 103
+    assert lib.fp8attn_version() == 104
 
 
 def test_status_strings(lib):
@@ -156,3 +156,12 @@ def test_attention_rejects_unusable_out(bad):
            "device": torch.empty((B, H, N, d), dtype=torch.bfloat16, device="meta")}[bad]
     with pytest.raises(ValueError):
         attention(q, q, q, out=out)
+
+
+def test_schedule_switch(lib):
+    """fp8attn_set_schedule returns the previous schedule and refuses unknown ones."""
+    from online_softmax_tcgen05_b200 import SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES
+    assert lib.fp8attn_set_schedule(SCHEDULE_TWO_TILES) == SCHEDULE_ONE_TILE
+    assert lib.fp8attn_set_schedule(SCHEDULE_ONE_TILE) == SCHEDULE_TWO_TILES
+    assert lib.fp8attn_set_schedule(7) == EINVAL
+    assert lib.fp8attn_set_schedule(SCHEDULE_ONE_TILE) == SCHEDULE_ONE_TILE

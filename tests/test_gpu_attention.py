@@ -686,3 +686,74 @@ def test_attention_rejects_mixed_devices():
         attention(q, q.cpu(), q)
     with pytest.raises(ValueError):
         attention(q, q, q, out=torch.empty((1, 1, 128, 64), dtype=torch.bfloat16))
+
+
+# ------------------------------------------------- two-tile schedule --------
+SCHED_CASES = [
+    # B, H, Hkv, N, d, block_n, causal, S, order, qk_bf16, denominator, o_f32
+    (1, 8, 2, 4096, 128, 128, 1, 256.0, 1, False, 0, False),   # GQA: head pairs
+    (1, 8, 2, 4096, 128, 128, 0, 1.0, 0, False, 0, True),
+    (2, 3, 3, 1000, 128, 128, 1, 256.0, 1, False, 0, True),    # MHA: tile pairs, odd tiles
+    (1, 2, 2, 1000, 128, 64, 1, 448.0, 0, False, 0, True),     # block_n 64, S = 448
+    (2, 4, 2, 520, 64, 64, 0, 300.0, 1, False, 0, False),      # d 64, S = 300
+    (1, 4, 1, 777, 64, 128, 1, 16.0, 0, False, 0, True),       # group 4, ragged
+    (1, 5, 1, 333, 128, 128, 1, 256.0, 1, False, 0, True),     # odd group: tile pairs
+    (1, 4, 2, 700, 128, 128, 1, 256.0, 1, True, 0, True),      # BF16 Q/K
+    (1, 2, 1, 700, 128, 128, 1, 448.0, 0, False, 1, True),     # cast-value denominator
+    (1, 2, 2, 100, 128, 128, 1, 256.0, 1, False, 0, True),     # one tile: B tile empty
+]
+
+
+@pytest.mark.parametrize("case", SCHED_CASES)
+def test_two_tile_schedule_equals_one_tile(case):
+    """The two-tile schedule (two query tiles per CTA, exponential turns) against
+    the default one-tile schedule: same O bit for bit, same counters and per-row
+    counts.  The one-tile kernel is the one checked against the oracle above."""
+    from online_softmax_tcgen05_b200 import SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES, set_schedule
+    B, H, Hkv, N, d, block_n, causal, S, order, qk_bf16, denom, f32 = case
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 9.0, seed=3000 + N + H)
+    ins = gpu_inputs_bf16(W) if qk_bf16 else gpu_inputs(W)
+    outs = []
+    try:
+        for sched in (SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES):
+            set_schedule(sched)
+            outs.append(run_gpu(ins, B, H, Hkv, N, d, causal, S, order, block_n, 4, f32,
+                                denominator=denom))
+    finally:
+        set_schedule(SCHEDULE_ONE_TILE)
+    (O1, t1, s1, r1), (O2, t2, s2, r2) = outs
+    assert np.array_equal(O1, O2, equal_nan=False), (case, np.abs(O1 - O2).max())
+    assert (t1, s1) == (t2, s2) and np.array_equal(r1, r2), case
+
+
+def test_two_tile_schedule_row_ranges():
+    """Query-row ranges with the two-tile schedule (a range of an odd number of
+    tiles leaves the second tile of the last pair outside the range): the rows
+    of each range equal the full launch's, the others stay untouched."""
+    import torch
+    from online_softmax_tcgen05_b200 import (O_F32, SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES,
+                                             fp8_attn_fwd_ex, set_schedule)
+    B, H, Hkv, N, d = 1, 4, 4, 1000, 128
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 8.0, seed=23)
+    ins = gpu_inputs(W)
+    (Qg, _), (Kg, _), (Vg, _) = ins
+    full, tot, sink_tot, crow = run_gpu(ins, B, H, Hkv, N, d, 1, 256.0, 1, 128, 4)
+    full = full.reshape(B, H, N, d)
+    try:
+        set_schedule(SCHEDULE_TWO_TILES)
+        O = torch.full((B, H, N, d), float("nan"), dtype=torch.float32, device=Qg.device)
+        ctr = torch.zeros(2, dtype=torch.int64, device=Qg.device)
+        done = np.zeros(N, dtype=bool)
+        for lo, hi in ((384, 640), (0, 128), (640, N), (128, 384)):
+            fp8_attn_fwd_ex(Qg, Kg, Vg, O, B=B, H=H, H_kv=Hkv, N=N, d=d, causal=1, S=256.0,
+                            kv_order=1, n_sink=4, o_dtype=O_F32, collapse_ctr=ctr[0:1],
+                            collapse_sink_ctr=ctr[1:2], q_begin=lo, q_end=hi)
+            torch.cuda.synchronize()
+            done[lo:hi] = True
+            Oc = O.cpu().numpy()
+            assert np.array_equal(Oc[:, :, done], full[:, :, done])
+            assert np.isnan(Oc[:, :, ~done]).all()
+        c = ctr.cpu().numpy()
+        assert int(c[0]) == tot and int(c[1]) == sink_tot
+    finally:
+        set_schedule(SCHEDULE_ONE_TILE)

@@ -75,3 +75,36 @@ def test_host_entry_reports_expired_wait_and_recovers():
                                    4)
     assert_o_close(O.numpy().reshape(-1, d), Oe, "host entry after timeout")
     plan.close()
+
+
+def test_expired_wait_with_two_tile_schedule():
+    """The same expired wait under the two-tile schedule, whose softmax warps
+    take turns on named barriers: the aborting warps keep taking their turns
+    (without touching TMEM), so the launch ends, reports the timeout, and the
+    next launch on the same context is correct."""
+    import torch
+    from online_softmax_tcgen05_b200 import (O_F32, SCHEDULE_ONE_TILE, SCHEDULE_TWO_TILES,
+                                             fp8_attn_fwd_ex, set_schedule)
+    B, H, N, d = 1, 1, 512, 128
+    W = workload.make_sink_workload(B, H, H, N, d, 4, 8.0, seed=9)
+    ins = gpu_inputs(W)
+    (q, Q8), (k, K8), (v, V8) = ins
+    O = torch.zeros((B, H, N, d), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        set_schedule(SCHEDULE_TWO_TILES)
+        fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=H, N=N, d=d, S=256.0, kv_order=1, n_sink=4,
+                        o_dtype=O_F32, status_word=status, timeout_ns=50_000_000,
+                        debug_skip_kv_step=2)
+        torch.cuda.synchronize()
+        word = int(status.item())
+        assert (word & ~0xFF) == 0x100 and (word & 0xFF) != 0, hex(word)
+        status.zero_()
+        fp8_attn_fwd_ex(q, k, v, O, B=B, H=H, H_kv=H, N=N, d=d, S=256.0, kv_order=1, n_sink=4,
+                        o_dtype=O_F32, status_word=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+    finally:
+        set_schedule(SCHEDULE_ONE_TILE)
+    Oe, _, _ = oracle.attn_emulate(Q8, K8, V8, B, H, H, N, d, 0, 1 / math.sqrt(d), 256.0, 1, 128, 4)
+    assert_o_close(O.cpu().numpy().reshape(-1, d), Oe, "two-tile schedule after timeout")
