@@ -257,6 +257,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     fa.load_library()
+    fa.set_schedule(fa.SCHEDULE_TWO_TILES if args.schedule == "two-tiles" else fa.SCHEDULE_ONE_TILE)
     import workload
     strong = args.shard == "heads"
     cfg = CFG_LONG if strong else CFG
@@ -373,6 +374,7 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e / e2e_steps, 3)},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
+        "kernel_schedule": args.schedule,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(W, cfg, n_rows=8192 if strong else 65536)
@@ -763,6 +765,9 @@ def main():
     ap.add_argument("--shard", choices=["replica", "heads"], default="replica",
                     help="replica: one independent prefill per rank (weak scaling); heads: "
                          "the long-context problem split by kv heads (strong scaling)")
+    ap.add_argument("--schedule", choices=["one-tile", "two-tiles"], default="one-tile",
+                    help="kernel schedule (fp8attn_set_schedule): one query tile per CTA "
+                         "(default) or two per CTA with turns on the exponential unit")
     ap.add_argument("--mode", choices=["full", "kernel"], default="full",
                     help="kernel: only the device-timed kernel loop (for profiling)")
     ap.add_argument("--report", choices=["collapse", "configs", "batched-orders", "e2e-timeline",
