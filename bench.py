@@ -143,7 +143,8 @@ KERNEL_SOURCES = ["online_softmax_tcgen05_b200/csrc/fp8_attn_fwd.cu",
                   "online_softmax_tcgen05_b200/csrc/attn_kernel.cuh",
                   "online_softmax_tcgen05_b200/csrc/sm100.cuh",
                   "online_softmax_tcgen05_b200/csrc/exp2_poly.cuh",
-                  "online_softmax_tcgen05_b200/csrc/row_max.cuh"]
+                  "online_softmax_tcgen05_b200/csrc/row_max.cuh",
+                  "online_softmax_tcgen05_b200/csrc/softmax_block.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_prefill_N32768.json")
 
 

@@ -17,7 +17,8 @@ LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libfp8attn.so")
 SOURCES = ["fp8_attn_fwd.cu", "fp8_attn_fwd_pair.cu", "fp8attn_abi.cu", "fp8attn_host.cu",
            "fp8attn_host_noalloc.cu"]
-HEADERS = ["attn_kernel.cuh", "abi_internal.h", "sm100.cuh", "exp2_poly.cuh", "row_max.cuh"]
+HEADERS = ["attn_kernel.cuh", "abi_internal.h", "sm100.cuh", "exp2_poly.cuh", "row_max.cuh",
+           "softmax_block.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]

@@ -38,10 +38,10 @@
 #include <cstdint>
 
 #include "attn_kernel.cuh"
-#include "exp2_poly.cuh"
 #include "fp8attn.h"
 #include "row_max.cuh"
 #include "sm100.cuh"
+#include "softmax_block.cuh"
 
 namespace fp8attn {
 
@@ -73,15 +73,6 @@ struct Smem {
   static constexpr uint32_t TMEM_COLS = 256;    // S: BN columns, O: D columns
   static_assert(BN + D <= (int)TMEM_COLS, "TMEM budget");
 };
-
-template <bool B>
-struct BoolTag {
-  static constexpr bool value = B;
-};
-
-__device__ __forceinline__ int kv_block_at(int t, int T, int order) {
-  return order == FP8ATTN_KV_FORWARD ? t : T - 1 - t;
-}
 
 // QB: bytes per Q / K element.  1: E4M3 Q and K, QK^T as kind::f8f6f4.
 // 2: BF16 Q and K, QK^T as kind::f16 (the "kernel-faithful" reading of the
@@ -338,110 +329,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       auto block_math = [&](auto plain_tag) {
         constexpr bool PLAIN = decltype(plain_tag)::value;
         if constexpr (!PLAIN) {
-          if (need_mask) {
-#pragma unroll
-            for (int j = 0; j < BN; ++j)
-              if (j0 + j > lim) s[j] = -INFINITY;
-          }
+          if (need_mask) mask_scores<BN>(s, j0, lim);
         }
         const float mx = row_max<BN>(s);
         m_new = fmaxf(m_run, mx * c);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
-        // 2^(s*c - m + log2S): packed FFMA2 for the argument, MUFU ex2, split row
-        // sums.  For S = 2^k (log2S = k) that is S*p and its row sum carries S;
-        // otherwise (log2S = 0) it is p, multiplied by S below.
+        // 2^(s*c - m + log2S): for S = 2^k (log2S = k) that is S*p and its row sum
+        // carries S; otherwise (log2S = 0) it is p, multiplied by S in the cast.
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
-        float2 acc8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < BN / 2; ++q) {
-          const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
-          if ((q & 7) < POLY_OF_8) {
-            const float2 e = exp2_poly2(y);
-            s[2 * q] = e.x;
-            s[2 * q + 1] = e.y;
-          } else {
-            s[2 * q] = ex2_approx(y.x);
-            s[2 * q + 1] = ex2_approx(y.y);
-          }
-          acc8[q & 7] = __fadd2_rn(acc8[q & 7], make_float2(s[2 * q], s[2 * q + 1]));
-        }
-#pragma unroll
-        for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) acc8[i] = __fadd2_rn(acc8[i], acc8[i + w]);
-        const float rowsum = acc8[0].x + acc8[0].y;
-        if constexpr (PLAIN) {
-          l = alpha * l + rowsum;
-        } else {
-          if (!p.denom_cast) l = alpha * l + rowsum;
-        }
-        // the E4M3 cast of S*p, four keys per word.  Blocks off the plain path
-        // form fl(s_mul * x): the method's FP32 product S*p when S is not a power
-        // of two, an exact multiply by 1 when S*p came out of the exponential.
-        const float2 sm2 = make_float2(p.s_mul, p.s_mul);
-#pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-          if constexpr (PLAIN) {
-            pw[q] = pack_e4m3x4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-          } else {
-            const float2 a = __fmul2_rn(make_float2(s[4 * q], s[4 * q + 1]), sm2);
-            const float2 b = __fmul2_rn(make_float2(s[4 * q + 2], s[4 * q + 3]), sm2);
-            pw[q] = pack_e4m3x4(a.x, a.y, b.x, b.y);
-          }
-        }
+        const float rowsum = exp2_rowsum<BN, POLY_OF_8, false>(s, c2, nm2);
+        if (PLAIN || !p.denom_cast) l = scale_add(alpha, l, rowsum);
+        cast_e4m3<BN, !PLAIN>(s, p.s_mul, pw);
         if constexpr (!PLAIN) {
-          if (p.denom_cast) {
-            // l from the cast values: an E4M3 magnitude's 7 bits placed at FP32 bit 20
-            // form a float exactly 2^-120 times the E4M3 value (subnormals included,
-            // as FP32 subnormals); sum those, then scale by 2^120 (exact).
-            float2 d4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int q = 0; q < BN / 4; ++q) {
-              const uint32_t w = pw[q];
-              const float2 lo = make_float2(__uint_as_float((w & 0x7Fu) << 20),
-                                            __uint_as_float((w & 0x7F00u) << 12));
-              const float2 hi = make_float2(__uint_as_float((w & 0x7F0000u) << 4),
-                                            __uint_as_float((w & 0x7F000000u) >> 4));
-              d4[q & 3] = __fadd2_rn(d4[q & 3], __fadd2_rn(lo, hi));
-            }
-            d4[0] = __fadd2_rn(__fadd2_rn(d4[0], d4[1]), __fadd2_rn(d4[2], d4[3]));
-            l = alpha * l + (d4[0].x + d4[0].y) * 0x1p120f;
-          }
+          if (p.denom_cast) l = scale_add(alpha, l, cast_value_sum<BN>(pw));
         }
         if constexpr (COUNT) {
-          // Collapse: a visible non-sink key whose E4M3 byte is zero.  P~ is never
-          // negative, so byte 0 <=> the cast flushed S*p to zero.
+          // Collapse: a visible non-sink key whose E4M3 byte is zero (P~ is never
+          // negative, so byte 0 <=> the cast flushed S*p to zero).  Blocks that
+          // hold a sink or a masked key count the keys n_sink <= j <= lim only.
           uint32_t cblk;
-          if (PLAIN || (j0 >= p.n_sink && !need_mask)) {
-            // Every byte is 0x00..0x7F (sign clear: S*p >= +0; a NaN casts to
-            // 0x7F), so w + 0x7F7F7F7F carries into no neighbour and sets bit 7
-            // of exactly the nonzero bytes; dp4a sums those four flags (x128).
-            uint32_t nz4[4] = {0, 0, 0, 0};
-#pragma unroll
-            for (int q = 0; q < BN / 4; ++q)
-              nz4[q & 3] = __dp4a((pw[q] + 0x7F7F7F7Fu) & 0x80808080u, 0x01010101u, nz4[q & 3]);
-            cblk = BN - (((nz4[0] + nz4[1]) + (nz4[2] + nz4[3])) >> 7);
-          } else {
-            // blocks that hold a sink or a masked key count only the lanes with
-            // n_sink <= j <= last visible key
-            uint32_t zacc = 0;
-            const int lo = max(p.n_sink - j0, 0), hi = min(lim - j0, BN - 1);   // block-local
-#pragma unroll
-            for (int q = 0; q < BN / 4; ++q) {
-              const uint32_t w = pw[q];
-              uint32_t y = ~(((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w | 0x7F7F7F7Fu);
-              const int a = lo - 4 * q, bq = hi - 4 * q;   // lanes a..bq of this word are valid
-              const uint32_t mlo = a <= 0 ? 0x80808080u : (a >= 4 ? 0u : 0x80808080u << (8 * a));
-              const uint32_t mhi = bq >= 3 ? 0x80808080u : (bq < 0 ? 0u : 0x80808080u >> (8 * (3 - bq)));
-              zacc += (y & mlo & mhi) >> 7;
-            }
-            cblk = (zacc * 0x01010101u) >> 24;   // byte lanes hold <= BN/4 each
-          }
+          if (PLAIN || (j0 >= p.n_sink && !need_mask))
+            cblk = zero_bytes_all<BN>(pw);
+          else
+            cblk = zero_bytes_range<BN>(pw, max(p.n_sink - j0, 0), min(lim - j0, BN - 1));
           cnt += cblk;
           if constexpr (!PLAIN) {
             if (j0 < p.n_sink) cnt_sink += cblk;
@@ -464,37 +375,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!ok) break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < BN / 16; ++q) {
-        const uint32_t dst = prow + ((q ^ pswz) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pw[4 * q]),
-                     "r"(pw[4 * q + 1]), "r"(pw[4 * q + 2]), "r"(pw[4 * q + 3])
-                     : "memory");
-      }
+      store_p_row<BN>(pw, prow, pswz);
       if (t > 0) {
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          // O *= alpha for this warp's 32 rows, 64 TMEM columns per round trip
-          const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-          for (int cc = 0; cc < D / 32; cc += 2) {
-            uint32_t o0[32], o1[32];
-            tmem_ld32(tO + 32 * cc, o0);
-            tmem_ld32(tO + 32 * cc + 32, o1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              float2 r0 = __fmul2_rn(make_float2(__uint_as_float(o0[k]), __uint_as_float(o0[k + 1])), a2);
-              float2 r1 = __fmul2_rn(make_float2(__uint_as_float(o1[k]), __uint_as_float(o1[k + 1])), a2);
-              o0[k] = __float_as_uint(r0.x);
-              o0[k + 1] = __float_as_uint(r0.y);
-              o1[k] = __float_as_uint(r1.x);
-              o1[k + 1] = __float_as_uint(r1.y);
-            }
-            tmem_st32(tO + 32 * cc, o0);
-            tmem_st32(tO + 32 * cc + 32, o1);
-          }
-          tmem_wait_st();
-        }
+        // O *= alpha for this warp's rows when one of their maxima rose
+        if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(tO, alpha);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -512,38 +396,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // multiply per element.  For S = 2^k, l already is the row sum of S*p
       // (s_mul = 1); otherwise the denominator is fl(S * l).  The cast-value row
       // sum carries S in its values.
-      const float inv_l = __frcp_rn(p.denom_cast ? l : l * p.s_mul);
+      const float inv_l = __frcp_rn(p.denom_cast ? l : __fmul_rn(l, p.s_mul));
       const bool live = row < p.N;
       const size_t obase = ((size_t)bh * p.N + (size_t)(live ? row : 0)) * D;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * cc, o);
-        tmem_wait_ld();
-        float v[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * inv_l;
-        if (live) {
-          if constexpr (OUT_BF16) {
-            uint32_t w[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              uint32_t bits;
-              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(bits) : "f"(v[2 * k + 1]), "f"(v[2 * k]));
-              w[k] = bits;
-            }
-            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + obase + 32 * cc);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              out[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-          } else {
-            float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.O) + obase + 32 * cc);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              out[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-          }
-        }
-      }
+      store_o_row<D, OUT_BF16>(tO, inv_l, live, p.O, obase);
       if constexpr (COUNT) {
         if (!live) cnt = cnt_sink = 0;   // padding rows past a ragged N
         if (p.rows && live) p.rows[(size_t)bh * p.N + row] = cnt;
