@@ -8,9 +8,14 @@
 // exchange, then rounded to FP32); 2^n is added to the exponent field.
 // Maximum relative error of the FP32 evaluation: 2.2e-7 (about 2 ulp).
 // x is clamped to >= -125 so that every result is a normal float; callers use
-// it for x <= 0, where the clamp only turns values below 2^-125 into 2^-125.
+// it for x <= 8, where the clamp only turns values below 2^-125 into 2^-125
+// (zero after any E4M3 cast, and below every FP32 row sum's last bit).  The
+// clamp maps a NaN x to -125: the softmax keeps NaN through its row maximum
+// instead (row_max.cuh), which makes every exponential of the row NaN.
 #pragma once
 #include <cuda_runtime.h>
+
+#include <cstdint>
 
 namespace fp8attn {
 
@@ -22,7 +27,13 @@ constexpr float EXP2_C4 = 0.009675540961325169f;
 constexpr float EXP2_C5 = 0.0013276472454890609f;
 constexpr float EXP2_ROUND = 12582912.0f;   // 1.5 * 2^23
 
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+// 2^x for a pair.  sc23 must hold 2^23: the exponent is added as
+// bits(p) + bits(x + 1.5*2^23) * 2^23 (mod 2^32; the low mantissa bits of the
+// sum hold n, the high bits shift out), an integer multiply-add, so that the
+// exponent step runs on the FMA pipe with the polynomial.  The caller passes
+// 2^23 as a run-time value so that it stays a multiply-add rather than a shift
+// on the integer ALU, which the softmax's cast and count already keep busy.
+__device__ __forceinline__ float2 exp2_poly2(float2 x, uint32_t sc23) {
   x.x = fmaxf(x.x, -125.f);
   x.y = fmaxf(x.y, -125.f);
   const float2 y = __fadd2_rn(x, make_float2(EXP2_ROUND, EXP2_ROUND));
@@ -33,9 +44,12 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   p = __ffma2_rn(p, f, make_float2(EXP2_C2, EXP2_C2));
   p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
   p = __ffma2_rn(p, f, make_float2(EXP2_C0, EXP2_C0));
-  // low mantissa bits of y hold n; shifting them into the exponent field adds n
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));
+  uint32_t rx, ry;
+  asm("mad.lo.u32 %0, %1, %2, %3;"
+      : "=r"(rx) : "r"(__float_as_uint(y.x)), "r"(sc23), "r"(__float_as_uint(p.x)));
+  asm("mad.lo.u32 %0, %1, %2, %3;"
+      : "=r"(ry) : "r"(__float_as_uint(y.y)), "r"(sc23), "r"(__float_as_uint(p.y)));
+  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 }  // namespace fp8attn

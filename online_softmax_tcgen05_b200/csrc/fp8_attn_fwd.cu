@@ -47,13 +47,6 @@ namespace fp8attn {
 
 constexpr int NSTAGE = 2;       // K/V ring depth
 constexpr int NTHREADS = 192;   // 4 softmax warps + TMA warp + MMA warp
-// Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
-// (exp2_poly.cuh) and the rest on MUFU ex2: the two units then share the
-// exponentials of the softmax.
-#ifndef FP8ATTN_POLY_OF_8
-#define FP8ATTN_POLY_OF_8 0
-#endif
-constexpr int POLY_OF_8 = FP8ATTN_POLY_OF_8;
 
 template <int D, int BN, int QB>
 struct Smem {
@@ -294,6 +287,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     const uint32_t tS = tmem_base + lane_off, tO = tmem_base + lane_off + BN;
     const float c = p.scale_log2;
+    const uint32_t sc23 = (uint32_t)(p.N > 0) << 23;   // 2^23, a run-time value (exp2_poly2)
     float m_run = -INFINITY, l = 0.f;
     uint32_t cnt = 0, cnt_sink = 0;
     bool ok = true;
@@ -332,13 +326,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (need_mask) mask_scores<BN>(s, j0, lim);
         }
         const float mx = row_max<BN>(s);
-        m_new = fmaxf(m_run, mx * c);
+        m_new = fmax_nan(m_run, mx * c);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
         // 2^(s*c - m + log2S): for S = 2^k (log2S = k) that is S*p and its row sum
         // carries S; otherwise (log2S = 0) it is p, multiplied by S in the cast.
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
-        const float rowsum = exp2_rowsum<BN, POLY_OF_8, false>(s, c2, nm2);
+        const float rowsum = exp2_rowsum<BN, PLAIN ? POLY_OF_8 : 0, false>(s, c2, nm2, sc23);
         if (PLAIN || !p.denom_cast) l = scale_add(alpha, l, rowsum);
         cast_e4m3<BN, !PLAIN>(s, p.s_mul, pw);
         if constexpr (!PLAIN) {

@@ -88,13 +88,6 @@ constexpr int TURN_SCOPE = FP8ATTN_TURN_SCOPE;
 #define FP8ATTN_EXP_SPLIT 0
 #endif
 constexpr bool EXP_SPLIT = FP8ATTN_EXP_SPLIT != 0;
-// Of every 8 pairs of keys in a row, this many take 2^x on the FMA pipe
-// (exp2_poly.cuh) and the rest on MUFU ex2 during a warp's turn, when the FMA
-// pipe is otherwise nearly idle.
-#ifndef FP8ATTN_PAIR_POLY_OF_8
-#define FP8ATTN_PAIR_POLY_OF_8 0
-#endif
-constexpr int PAIR_POLY_OF_8 = FP8ATTN_PAIR_POLY_OF_8;
 
 // Waits of this kernel's roles: with a suspend-time hint (ns) a waiting warp
 // sleeps between probes instead of issuing them back to back.
@@ -385,6 +378,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t my_turn = (x == 0 ? TURN_A : TURN_B) + quarter;
     const uint32_t other_turn = (x == 0 ? TURN_B : TURN_A) + quarter;
     const float c = p.scale_log2;
+    const uint32_t sc23 = (uint32_t)(p.N > 0) << 23;   // 2^23, a run-time value (exp2_poly2)
     float m_run = -INFINITY, l = 0.f;
     uint32_t cnt = 0, cnt_sink = 0;
     const uint32_t prow = sP + x * BM * BN + (r >> 3) * (8 * BN) + (r & 7) * BN;
@@ -428,7 +422,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (lane == 0) mbar_arrive(bar_s_free(x));
         if (need_mask) mask_scores<BN>(s, j0, lim);
         const float mx = row_max<BN>(s);
-        m_new = fmaxf(m_run, mx * c);
+        m_new = fmax_nan(m_run, mx * c);
         alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
       }
 
@@ -441,7 +435,8 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
         constexpr bool PLAIN = decltype(plain_tag)::value;
         const float m_use = (m_turn == -INFINITY) ? 0.f : m_turn;
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
-        const float rowsum = exp2_rowsum<BN, PAIR_POLY_OF_8, EXP_SPLIT>(s, c2, nm2);
+        const float rowsum =
+            exp2_rowsum<BN, PLAIN ? POLY_OF_8 : 0, EXP_SPLIT>(s, c2, nm2, sc23);
         if constexpr (TURN_SCOPE == 1) {
           if (x == 0 || t + 1 < T) turn_pass(other_turn, rowsum);
         }

@@ -21,6 +21,15 @@
 
 namespace fp8attn {
 
+// Of every 8 pairs of keys in a row of a plain block (no masked key), this many
+// take 2^x on the FMA pipe (exp2_poly.cuh) and the rest on MUFU ex2: the two
+// units then share the exponentials of the softmax.  Both kernel schedules use
+// the same split, so that they compute the same values.
+#ifndef FP8ATTN_POLY_OF_8
+#define FP8ATTN_POLY_OF_8 2
+#endif
+constexpr int POLY_OF_8 = FP8ATTN_POLY_OF_8;
+
 template <bool B>
 struct BoolTag {
   static constexpr bool value = B;
@@ -50,10 +59,12 @@ __device__ __forceinline__ void mask_scores(float* s, int j0, int lim) {
 // s[j] <- 2^(s[j] * c + nm) in place (c2 = (c, c), nm2 = (nm, nm)); returns the
 // FP32 row sum of the results.  The argument is one packed FFMA2 per pair of keys
 // and the exponential MUFU ex2, except for POLY of every 8 pairs, which take the
-// FMA-pipe 2^x of exp2_poly.cuh.  The sum runs in 8 packed partial sums, reduced
-// by a fixed tree.  SPLIT issues every exponential before the first sum.
+// FMA-pipe 2^x of exp2_poly.cuh (finite arguments only: -inf, a masked key, needs
+// the MUFU path); sc23 = 2^23 as a run-time value (exp2_poly2).  The sum runs in 8
+// packed partial sums, reduced by a fixed tree.  SPLIT issues every exponential
+// before the first sum.
 template <int BN, int POLY, bool SPLIT>
-__device__ __forceinline__ float exp2_rowsum(float* s, float2 c2, float2 nm2) {
+__device__ __forceinline__ float exp2_rowsum(float* s, float2 c2, float2 nm2, uint32_t sc23) {
   float2 acc8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc8[i] = make_float2(0.f, 0.f);
@@ -72,7 +83,7 @@ __device__ __forceinline__ float exp2_rowsum(float* s, float2 c2, float2 nm2) {
     for (int q = 0; q < BN / 2; ++q) {
       const float2 y = __ffma2_rn(make_float2(s[2 * q], s[2 * q + 1]), c2, nm2);
       if ((q & 7) < POLY) {
-        const float2 e = exp2_poly2(y);
+        const float2 e = exp2_poly2(y, sc23);
         s[2 * q] = e.x;
         s[2 * q + 1] = e.y;
       } else {

@@ -757,3 +757,41 @@ def test_two_tile_schedule_row_ranges():
         assert int(c[0]) == tot and int(c[1]) == sink_tot
     finally:
         set_schedule(SCHEDULE_ONE_TILE)
+
+
+@pytest.mark.parametrize("schedule", [0, 1])
+@pytest.mark.parametrize("order", [0, 1])
+def test_nan_input_reaches_exactly_the_rows_that_see_it(schedule, order):
+    """A NaN E4M3 byte in K makes the O rows of every query that sees that key
+    NaN (both on a key whose exponential takes the FMA-pipe 2^x and on one that
+    takes MUFU ex2), a NaN byte in Q makes its own row NaN, and every other row
+    equals the clean run bit for bit (with the same counts per row)."""
+    import torch
+    from online_softmax_tcgen05_b200 import SCHEDULE_ONE_TILE, set_schedule
+    B, H, Hkv, N, d = 1, 2, 1, 1000, 128
+    W = workload.make_sink_workload(B, H, Hkv, N, d, 4, 8.0, seed=41)
+    ins = gpu_inputs(W)
+    (Qg, Q8), (Kg, K8), (Vg, V8) = ins
+    # key 300: key pair 150, position 150 % 8 = 6 of its group of 8 pairs (MUFU);
+    # key 513: pair 256, position 0 (the FMA-pipe positions are the first ones)
+    kbad, qbad = (300, 513), 100
+    K2, Q2 = Kg.clone(), Qg.clone()
+    for j in kbad:
+        K2[0, 0, j, 5] = 0x7F
+    Q2[0, 1, qbad, 9] = 0x7F
+    ins2 = ((Q2, Q8), (K2, K8), (Vg, V8))
+    try:
+        set_schedule(schedule)
+        clean = run_gpu(ins, B, H, Hkv, N, d, 1, 256.0, order, 128, 4)
+        bad = run_gpu(ins2, B, H, Hkv, N, d, 1, 256.0, order, 128, 4)
+    finally:
+        set_schedule(SCHEDULE_ONE_TILE)
+    Oc, Ob = clean[0].reshape(H, N, d), bad[0].reshape(H, N, d)
+    rc, rb = clean[3].reshape(H, N), bad[3].reshape(H, N)
+    sees = np.zeros((H, N), dtype=bool)
+    sees[:, min(kbad):] = True          # causal: query i sees key j iff j <= i
+    sees[1, qbad] = True
+    assert np.isnan(Ob[sees]).all()
+    assert np.isfinite(Oc).all()
+    assert np.array_equal(Ob[~sees], Oc[~sees])
+    assert np.array_equal(rb[~sees], rc[~sees])
