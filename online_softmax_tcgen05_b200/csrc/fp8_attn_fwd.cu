@@ -302,9 +302,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int j0 = kv_block_at(t, T, p.kv_order) * BN;
       tc_fence_after();
       uint32_t sr[BN];
+      if constexpr (COUNT && BN == 128) {
+        // one 128-column load: timed 1.7-1.9% faster than four 32-column loads in
+        // the counting kernel and 2.5-3% slower in the plain one (same values)
+        tmem_ld128(tS, *reinterpret_cast<uint32_t(*)[128]>(&sr[0]));
+      } else {
 #pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc)
-        tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+        for (int cc = 0; cc < BN / 32; ++cc)
+          tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+      }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
