@@ -413,9 +413,15 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
       uint32_t pw[BN / 4];
       {
         tc_fence_after();
+        if constexpr (COUNT && BN == 128) {
+          // one 128-column load in the counting kernel (as in the one-tile kernel;
+          // timed 0.9-2.7% faster here, the plain kernel unchanged)
+          tmem_ld128(tS, *reinterpret_cast<uint32_t(*)[128]>(&sr[0]));
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc)
-          tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+          for (int cc = 0; cc < BN / 32; ++cc)
+            tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+        }
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
