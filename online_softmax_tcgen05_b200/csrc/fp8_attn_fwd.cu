@@ -338,9 +338,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // 2^(s*c - m + log2S): for S = 2^k (log2S = k) that is S*p and its row sum
         // carries S; otherwise (log2S = 0) it is p, multiplied by S in the cast.
         const float2 c2 = make_float2(c, c), nm2 = make_float2(p.log2S - m_use, p.log2S - m_use);
-        const float rowsum = exp2_rowsum<BN, PLAIN ? POLY_OF_8 : 0, false>(s, c2, nm2, sc23);
+        uint32_t zeros_plain = 0;   // the plain counting body's zero bytes
+        float rowsum;
+        if constexpr (PLAIN && COUNT) {
+          rowsum = exp_cast_count_plain<BN, POLY_OF_8>(s, c2, nm2, sc23, pw, &zeros_plain);
+        } else {
+          rowsum = exp2_rowsum<BN, PLAIN ? POLY_OF_8 : 0, false>(s, c2, nm2, sc23);
+          cast_e4m3<BN, !PLAIN>(s, p.s_mul, pw);
+        }
         if (PLAIN || !p.denom_cast) l = scale_add(alpha, l, rowsum);
-        cast_e4m3<BN, !PLAIN>(s, p.s_mul, pw);
         if constexpr (!PLAIN) {
           if (p.denom_cast) l = scale_add(alpha, l, cast_value_sum<BN>(pw));
         }
@@ -349,7 +355,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // negative, so byte 0 <=> the cast flushed S*p to zero).  Blocks that
           // hold a sink or a masked key count the keys n_sink <= j <= lim only.
           uint32_t cblk;
-          if (PLAIN || (j0 >= p.n_sink && !need_mask))
+          if constexpr (PLAIN)
+            cblk = zeros_plain;
+          else if (j0 >= p.n_sink && !need_mask)
             cblk = zero_bytes_all<BN>(pw);
           else
             cblk = zero_bytes_range<BN>(pw, max(p.n_sink - j0, 0), min(lim - j0, BN - 1));
