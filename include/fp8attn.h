@@ -32,6 +32,9 @@
  * the same real numbers, exact scaling.  For any other S it forms the FP32
  * product fl(S * p_j) that is cast, sums the p_j, and divides by fl(S * l).
  * Causal: key j is visible to query i iff j <= i (square prefill, no offset).
+ * NaN inputs: a NaN byte in Q or K makes every O row that sees it NaN (the row
+ * maximum keeps NaN, so all of that row's exponentials are NaN from that block
+ * on); rows that do not see it are unaffected.
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller (except Q, K, V, O
